@@ -1,0 +1,585 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise FP8 weight quantizer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload qwen3_8b_model|qwen3_8b_layer|moe_layer|small]
+                    [--path auto|vector|tma|generic]
+
+A step is one pass of the whole quantizer over the workload: by default the
+full Qwen3-8B-shaped weight set (36 layers x q,k,v,o,gate,up,down = 252 bf16
+tensors, 6.95e9 elements, 13.9 GB in + 6.95 GB out) quantized to e4m3fn with
+128x128 blocks in ONE grouped call of the C ABI (fp8bq_quantize_batched).
+
+Metric: GB/s of algorithmic bytes (input read + e4m3 write + fp32 descales),
+whole job over all ranks, timed with CUDA events on the launching stream, the
+inputs already resident in HBM; the inputs (13.9 GB) are far larger than L2
+(126 MB), so no flush is needed between steps.  `e2e` is the same metric
+with the inputs in pinned host memory and the outputs copied back to host
+memory inside the timed region, one C-ABI call per layer, the copies of
+neighbouring layers overlapping the compute.
+
+N > 1 (torchrun, one process per GPU): every rank quantizes its own replica of
+the weight set (weak scaling; no collective on the data path; the host inputs
+are generated once per node into shared memory).  Timing is the max over
+ranks.
+
+--impl reference times the CPU oracle (single thread) on a bounded sample of
+the same workload: one tensor per step, cycling through the weight set.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import hashlib
+import json
+import os
+import platform
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "blockwise FP8 quant GB/s (bytes in+out) and % of B200 HBM peak, 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["blockwise_fp8_weight_b200/csrc/fp8bq_kernels.cu",
+                  "blockwise_fp8_weight_b200/csrc/fp8bq_device.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+PATHS = {"auto": 0, "vector": 1, "tma": 2, "generic": 3}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+
+
+def dist_env() -> tuple[int, int, int]:
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+class Dist:
+    """Process-group plumbing: barrier and max-over-ranks of a scalar."""
+
+    def __init__(self, world: int, backend: str, device=None):
+        self.world = world
+        self.device = device
+        if world > 1:
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+            self.dist = dist
+
+    def barrier(self):
+        if self.world > 1:
+            if self.device is not None:
+                self.dist.barrier(device_ids=[self.device.index])
+            else:
+                self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=self.device or "cpu")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            self.dist.destroy_process_group()
+
+
+def aggregate(bytes_per_step: int, steps: int, world: int, max_elapsed_s: float) -> float:
+    """Whole-job GB/s: bytes every rank moved over all timed steps / slowest rank's time."""
+    return bytes_per_step * steps * world / max_elapsed_s / 1e9
+
+
+# ------------------------------------------------------------------ workload
+
+
+def workload(name: str):
+    from synth import workloads as W
+    if name == "qwen3_8b_model":
+        return W.qwen3_8b_model(), ("Qwen3-8B-shaped full weight set: 36 layers x (q,k,v,o,"
+                                    "gate,up,down) bf16, block 128x128, one grouped launch")
+    if name == "qwen3_8b_layer":
+        return W.qwen3_8b_layer(0, seed=1), ("one Qwen3-8B-shaped layer: 7 bf16 linear weights, "
+                                             "block 128x128, one grouped launch")
+    if name == "moe_layer":
+        return W.moe_layer(0), ("one Qwen3-30B-A3B-style MoE layer: q,k,v,o + 128-expert w13 "
+                                "and w2 stacks, bf16, block 128x128, one grouped launch")
+    if name == "small":
+        return W.small(), "256x384 bf16, 2x3 blocks of 128x128"
+    raise SystemExit(f"unknown workload {name}")
+
+
+def layers_of(specs) -> list[list[int]]:
+    """Group tensor indices by layer (consecutive) for the per-layer e2e pipeline."""
+    groups: list[list[int]] = []
+    last = object()
+    for i, sp in enumerate(specs):
+        key = sp.meta.get("layer", 0)
+        if key != last:
+            groups.append([])
+            last = key
+        groups[-1].append(i)
+    return groups
+
+
+def align(v: int, a: int) -> int:
+    return (v + a - 1) // a * a
+
+
+class Layout:
+    """Byte offsets of every tensor in the packed input / output buffers."""
+
+    def __init__(self, specs):
+        self.x_off, self.y_off, self.s_off = [], [], []
+        xo = yo = so = 0
+        for sp in specs:
+            self.x_off.append(xo)
+            self.y_off.append(yo)
+            self.s_off.append(so)
+            xo = align(xo + sp.numel_storage * sp.elem_bytes, 256)
+            yo = align(yo + sp.numel, 256)
+            so = align(so + sp.nblocks * 4, 256)
+        self.x_bytes, self.y_bytes, self.s_bytes = xo, yo, so
+
+
+def spec_digest(specs) -> str:
+    h = hashlib.sha256()
+    h.update(open(os.path.join(ROOT, "synth", "synth.c"), "rb").read())
+    h.update(open(os.path.join(ROOT, "synth", "workloads.py"), "rb").read())
+    for sp in specs:
+        h.update(repr((sp.name, sp.M, sp.N, sp.batch, sp.row_stride, sp.dtype, sp.seed,
+                       sp.tensor_id)).encode())
+    return h.hexdigest()[:16]
+
+
+def host_inputs(specs, lay: Layout, local_rank: int, dist: Dist, tag: str):
+    """Generate the packed host inputs once per node into /dev/shm (shared by the
+    ranks of a replica run); returns a writable numpy memmap."""
+    from synth import workloads as W
+    shm = "/dev/shm" if os.path.isdir("/dev/shm") else "/tmp"
+    path = os.path.join(shm, f"fp8bq_bench_{tag}_{spec_digest(specs)}.bin")
+    done = path + ".done"
+    if local_rank == 0 and not os.path.exists(done):
+        mm = np.memmap(path, dtype=np.uint8, mode="w+", shape=(lay.x_bytes,))
+        base = mm.ctypes.data
+        for sp, off in zip(specs, lay.x_off):
+            W.materialize_into(sp, base + off)
+        mm.flush()
+        del mm
+        open(done, "w").write("ok")
+    dist.barrier()
+    return np.memmap(path, dtype=np.uint8, mode="r+", shape=(lay.x_bytes,)), path
+
+
+# ------------------------------------------------------------------ measurement helpers
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
+               0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
+               0x200: "display_clock_setting"}
+
+    def __init__(self, torch_device, period_s=0.005):
+        self.period = period_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            p = torch.cuda.get_device_properties(torch_device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _reasons_now(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self._reasons_now()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self) -> dict:
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+
+
+def measured_peak() -> tuple[float, str]:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        v = float(json.load(open(p))["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_digest() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(workload_name: str, path: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    try:
+        rec = json.load(open(TRAFFIC_FILE))
+    except Exception:
+        return None
+    for r in rec.get("records", []):
+        if (r.get("workload") == workload_name and r.get("path") == path
+                and r.get("kernel_sources_sha256_16") == kernel_digest()):
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+# ------------------------------------------------------------------ arms
+
+
+def run_reference(args) -> None:
+    rank, _local, world = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from synth import workloads as W
+    specs, desc = workload(args.workload)
+    order = list(range(len(specs)))
+    total_bytes = 0
+    elapsed = 0.0
+    for step in range(args.warmup + args.steps):
+        sp = specs[order[step % len(order)]]
+        x = W.materialize(sp)
+        t0 = time.perf_counter()
+        for b in range(sp.batch):
+            xb = x[b * sp.batch_stride:(b + 1) * sp.batch_stride]
+            oracle.quantize(xb, sp.M, sp.N, sp.row_stride, *sp.block)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            total_bytes += sp.algorithmic_bytes
+            elapsed += dt
+    value = total_bytes / elapsed / 1e9
+    per_step = sum(sp.algorithmic_bytes for sp in specs)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_step / (value * 1e9) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": desc, "name": args.workload, "block": [128, 128]},
+        "cpu_baseline": {"kind": "oracle", "value": value, "unit": "GB/s", "cores": 1,
+                         "sample": f"one tensor of the workload per step, cycling from the "
+                                   f"first; {args.steps} timed tensors after {args.warmup} warm-up; "
+                                   f"single-threaded C oracle; {platform.processor() or 'cpu'}"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "ms_per_step extrapolates the sampled rate to the whole workload",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def build_descs(specs, lay: Layout, x_base: int, y_base: int, s_base: int, idx=None):
+    import blockwise_fp8_weight_b200 as fq
+    idx = range(len(specs)) if idx is None else idx
+    arr = (fq.fp8bq_desc * len(idx))()
+    for j, i in enumerate(idx):
+        sp = specs[i]
+        gm, gn = sp.grid
+        d = arr[j]
+        d.x = x_base + lay.x_off[i]
+        d.y_u8 = y_base + lay.y_off[i]
+        d.descale_f32 = s_base + lay.s_off[i]
+        d.M, d.N, d.ld, d.batch = sp.M, sp.N, sp.row_stride, sp.batch
+        d.x_batch_stride = sp.batch_stride
+        d.y_batch_stride = sp.M * sp.N
+        d.s_batch_stride = gm * gn
+        d.dtype_in = fq.FP8BQ_BF16 if sp.dtype == "bf16" else fq.FP8BQ_F32
+        d.block_m, d.block_n = sp.block
+        d.reserved = 0
+    return arr
+
+
+def count_launches(arr) -> int:
+    import blockwise_fp8_weight_b200 as fq
+    groups: dict = {}
+    for d in arr:
+        p = fq.fp8bq_path_for(d)
+        key = (p, d.dtype_in, d.block_m if p != 3 else 0, d.block_n if p != 3 else 0)
+        groups[key] = groups.get(key, 0) + 1
+    return sum(-(-n // (128 if k[0] == 2 else 320)) for k, n in groups.items())
+
+
+def cpu_baseline(specs, host: np.ndarray, lay: Layout, seconds: float) -> dict:
+    """The oracle as it stands, single-threaded, over whole tensors from the start
+    of the workload until about `seconds` of CPU time has been spent."""
+    import oracle
+    done_bytes, done = 0, []
+    t0 = time.perf_counter()
+    for i, sp in enumerate(specs):
+        x = host[lay.x_off[i]:lay.x_off[i] + sp.numel_storage * sp.elem_bytes].view(sp.np_dtype)
+        for b in range(sp.batch):
+            xb = np.ascontiguousarray(x[b * sp.batch_stride:(b + 1) * sp.batch_stride])
+            oracle.quantize(xb, sp.M, sp.N, sp.row_stride, *sp.block)
+        done_bytes += sp.algorithmic_bytes
+        done.append(sp.name)
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    cpu = platform.processor() or ""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                cpu = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"value": done_bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {len(done)} tensors of the workload ({done[0]} .. {done[-1]}), "
+                      f"{done_bytes / 1e9:.2f} GB moved in {dt:.1f} s; host {cpu}, "
+                      f"nproc {os.cpu_count()}"}
+
+
+def run_ours(args) -> None:
+    import torch
+    import blockwise_fp8_weight_b200 as fq
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = Dist(world, "nccl", dev)
+    specs, wl_desc = workload(args.workload)
+    lay = Layout(specs)
+    bytes_per_step = sum(sp.algorithmic_bytes for sp in specs)
+    elements = sum(sp.numel for sp in specs)
+
+    host, shm_path = host_inputs(specs, lay, local_rank, dist, args.workload)
+    cudart = torch.cuda.cudart()
+    hptr = host.ctypes.data
+    reg = cudart.cudaHostRegister(hptr, lay.x_bytes, 0)
+    pinned_in = int(reg) == 0
+    host_t = torch.from_numpy(host)
+
+    x_dev = torch.empty(lay.x_bytes, dtype=torch.uint8, device=dev)
+    x_dev.copy_(host_t, non_blocking=False)
+    y_dev = torch.empty(lay.y_bytes, dtype=torch.uint8, device=dev)
+    s_dev = torch.empty(lay.s_bytes, dtype=torch.uint8, device=dev)
+    table = build_descs(specs, lay, x_dev.data_ptr(), y_dev.data_ptr(), s_dev.data_ptr())
+    n = len(table)
+    assert fq.fp8bq_set_path(PATHS[args.path]) == fq.FP8BQ_OK
+    launches = count_launches(table)
+    L = fq.lib()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        st = L.fp8bq_quantize_batched(table, n, sh)
+        if st != 0:
+            raise RuntimeError(fq.fp8bq_status_string(st))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    fq.check(fq.fp8bq_sync_status(stream), "warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    dist.barrier()
+    fq.check(fq.fp8bq_sync_status(stream), "timed steps")
+    elapsed_s = t_start.elapsed_time(t_end) / 1e3
+    step_s = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    max_elapsed = dist.max(elapsed_s)
+    value = aggregate(bytes_per_step, args.steps, world, max_elapsed)
+
+    # ---- end to end: inputs from pinned host memory, outputs back to host memory
+    y_host = torch.empty(lay.y_bytes, dtype=torch.uint8, pin_memory=True)
+    s_host = torch.empty(lay.s_bytes, dtype=torch.uint8, pin_memory=True)
+    groups = layers_of(specs)
+    tables = [build_descs(specs, lay, x_dev.data_ptr(), y_dev.data_ptr(), s_dev.data_ptr(), g)
+              for g in groups]
+    s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+
+    def rng(off, sizes, g):
+        lo = off[g[0]]
+        hi = off[g[-1]] + sizes(g[-1])
+        return lo, hi
+
+    def e2e_step():
+        main = torch.cuda.current_stream(dev)
+        go = torch.cuda.Event()
+        go.record(main)
+        done = []
+        for gi, g in enumerate(groups):
+            xl, xh = rng(lay.x_off, lambda i: specs[i].numel_storage * specs[i].elem_bytes, g)
+            yl, yh = rng(lay.y_off, lambda i: specs[i].numel, g)
+            sl, shh = rng(lay.s_off, lambda i: specs[i].nblocks * 4, g)
+            s_in.wait_event(go)
+            with torch.cuda.stream(s_in):
+                x_dev[xl:xh].copy_(host_t[xl:xh], non_blocking=True)
+                e_in = torch.cuda.Event()
+                e_in.record(s_in)
+            s_cmp.wait_event(e_in)
+            st = L.fp8bq_quantize_batched(tables[gi], len(tables[gi]),
+                                          ctypes.c_void_p(s_cmp.cuda_stream))
+            if st != 0:
+                raise RuntimeError(fq.fp8bq_status_string(st))
+            e_c = torch.cuda.Event()
+            e_c.record(s_cmp)
+            s_out.wait_event(e_c)
+            with torch.cuda.stream(s_out):
+                y_host[yl:yh].copy_(y_dev[yl:yh], non_blocking=True)
+                s_host[sl:shh].copy_(s_dev[sl:shh], non_blocking=True)
+                e_o = torch.cuda.Event()
+                e_o.record(s_out)
+            done.append(e_o)
+        for e in done:
+            main.wait_event(e)
+
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    e2e_step()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    fq.check(fq.fp8bq_sync_status(), "e2e steps")
+    e2e_elapsed = dist.max(e0.elapsed_time(e1) / 1e3)
+    e2e_value = aggregate(bytes_per_step, e2e_steps, world, e2e_elapsed)
+    h2d = sum(sp.numel_storage * sp.elem_bytes for sp in specs)
+    d2h = sum(sp.numel + sp.nblocks * 4 for sp in specs)
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        cpu = cpu_baseline(specs, host, lay, args.cpu_seconds)
+
+    peak, peak_kind = measured_peak()
+    launch_s = float(np.mean(step_s)) / max(launches, 1)
+    achieved = bytes_per_step / max(launches, 1) / launch_s / 1e9
+    traffic = traffic_for(args.workload, args.path)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": max_elapsed / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl_desc, "name": args.workload, "tensors": len(specs),
+                       "elements": elements, "bytes_per_step": bytes_per_step,
+                       "block": [128, 128], "input_dtype": "bf16", "output_dtype": "e4m3fn",
+                       "path": args.path, "parallelism": f"replicas x{world}",
+                       "l2": "no flush: inputs per step exceed the 126 MB L2 by >100x"
+                       if lay.x_bytes > 1 << 30 else "inputs L2-resident: latency-bound case",
+                       "pct_hbm_peak": value / world / peak * 100.0,
+                       "elements_per_s": elements * args.steps * world / max_elapsed},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                         if peak_kind == "measured" else "fallback 6650 GB/s",
+                         "kernel_launches_per_step": launches,
+                         "avg_launch_ms": launch_s * 1e3},
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps, "pinned_input": pinned_in,
+                    "ms_per_step": e2e_elapsed / e2e_steps * 1e3},
+            "gpu_launches": launches * args.steps,
+            "clocks": clk.summary(),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+
+    fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
+    if pinned_in:
+        cudart.cudaHostUnregister(hptr)
+    del host_t, host
+    dist.barrier()
+    if local_rank == 0 and not args.keep_inputs:
+        for p in (shm_path, shm_path + ".done"):
+            try:
+                os.remove(p)
+            except OSError:
+                pass
+    dist.close()
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen3_8b_model",
+                    choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small"])
+    ap.add_argument("--path", choices=list(PATHS), default="auto")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU time spent on the oracle baseline (0 = skip)")
+    ap.add_argument("--keep-inputs", action="store_true",
+                    help="keep the generated host inputs in /dev/shm for the next run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    _rank, _local, world = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N > 1 needs torchrun with N processes")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,268 @@
+"""Blockwise FP8 (float8_e4m3fn) weight quantizer for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of the C ABI in ``include/fp8bq.h`` (library
+``libfp8bq.so``, built in-tree by ``blockwise_fp8_weight_b200.build``).  The
+functions named ``fp8bq_*`` mirror the C entry points one to one and only
+marshal arguments; every step of the quantization runs in the library's CUDA
+kernels.  There is no CPU or PyTorch fallback: if the library cannot be
+loaded, every call raises.
+
+On top of the raw entry points, two conveniences keep the call shapes of the
+pages' Python API (verl docs "fp8_kernel.py -- FP8 量化内核", section 1 and
+"vllm_fp8_utils.py", section 3):
+
+    scaled_fp8_blockwise(data_hp, weight_block_size) -> (fp8_data, descale)
+    quant_weights(named_weights, weight_block_size)  -> [(name, fp8), (name + "_scale_inv", s), ...]
+
+They allocate the outputs with PyTorch (device memory and streams are
+PyTorch's job here) and hand the pointers to the library.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Iterable, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfp8bq.so")
+
+# fp8bq_dtype
+FP8BQ_BF16 = 0
+FP8BQ_F32 = 1
+# fp8bq_status
+FP8BQ_OK = 0
+FP8BQ_ERR_NULL = 1
+FP8BQ_ERR_SHAPE = 2
+FP8BQ_ERR_BLOCK = 3
+FP8BQ_ERR_DTYPE = 4
+FP8BQ_ERR_OVERLAP = 5
+FP8BQ_ERR_DEVICE = 6
+FP8BQ_ERR_DEVICE_TIMEOUT = 7
+FP8BQ_ERR_ALIGN = 8
+FP8BQ_ERR_ARG = 9
+# fp8bq_path
+FP8BQ_PATH_AUTO = 0
+FP8BQ_PATH_VECTOR = 1
+FP8BQ_PATH_TMA = 2
+FP8BQ_PATH_GENERIC = 3
+FP8BQ_INJECT_DROP_FIRST_LOAD = 1
+
+DEFAULT_BLOCK = (128, 128)
+
+
+class fp8bq_desc(ctypes.Structure):
+    """Mirror of ``struct fp8bq_desc`` (96 bytes)."""
+    _fields_ = [
+        ("x", ctypes.c_void_p),
+        ("y_u8", ctypes.c_void_p),
+        ("descale_f32", ctypes.c_void_p),
+        ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("ld", ctypes.c_int64),
+        ("batch", ctypes.c_int64),
+        ("x_batch_stride", ctypes.c_int64),
+        ("y_batch_stride", ctypes.c_int64),
+        ("s_batch_stride", ctypes.c_int64),
+        ("dtype_in", ctypes.c_int32),
+        ("block_m", ctypes.c_int32), ("block_n", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class Fp8bqError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        msg = fp8bq_status_string(status)
+        super().__init__(f"{what}: {msg}" if what else msg)
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libfp8bq.so`` (building it first with nvcc if it is missing or
+    older than its sources).  Raises if it cannot be built or loaded."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            from . import build as _build
+            if not _build.up_to_date():
+                _build.build()
+            L = ctypes.CDLL(LIB_PATH)
+            vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            L.fp8bq_quantize.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, vp, vp]
+            L.fp8bq_quantize.restype = i32
+            L.fp8bq_quantize_batched.argtypes = [ctypes.POINTER(fp8bq_desc), i32, vp]
+            L.fp8bq_quantize_batched.restype = i32
+            L.fp8bq_status_string.argtypes = [i32]
+            L.fp8bq_status_string.restype = ctypes.c_char_p
+            L.fp8bq_sync_status.argtypes = [vp]
+            L.fp8bq_sync_status.restype = i32
+            L.fp8bq_version.argtypes = []
+            L.fp8bq_version.restype = i32
+            L.fp8bq_set_path.argtypes = [i32]
+            L.fp8bq_set_path.restype = i32
+            L.fp8bq_get_path.argtypes = []
+            L.fp8bq_get_path.restype = i32
+            L.fp8bq_path_for.argtypes = [ctypes.POINTER(fp8bq_desc)]
+            L.fp8bq_path_for.restype = i32
+            L.fp8bq_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.fp8bq_debug_set_wait_limit_ns.restype = i32
+            L.fp8bq_debug_set_inject.argtypes = [ctypes.c_uint32]
+            L.fp8bq_debug_set_inject.restype = i32
+            _lib = L
+    return _lib
+
+
+def _ptr(a) -> int:
+    """Pointer value of an int, None, or a tensor-like with data_ptr()."""
+    if a is None:
+        return 0
+    if isinstance(a, int):
+        return a
+    return int(a.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        if not torch.cuda.is_available():
+            return 0  # no device: the library reports FP8BQ_ERR_DEVICE itself
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+# ----------------------------------------------------------------- C entry points
+
+
+def fp8bq_quantize(x, dtype_in: int, M: int, N: int, ld: int, block_m: int, block_n: int,
+                   y_u8, descale_f32, stream=None) -> int:
+    """``fp8bq_quantize`` of the C ABI; pointers may be ints or tensors.
+    Returns the fp8bq_status code."""
+    return lib().fp8bq_quantize(_ptr(x), dtype_in, M, N, ld, block_m, block_n, _ptr(y_u8),
+                                _ptr(descale_f32), _stream(stream))
+
+
+def fp8bq_quantize_batched(desc_table: Sequence[fp8bq_desc] | ctypes.Array, n_tensors=None,
+                           stream=None) -> int:
+    """``fp8bq_quantize_batched`` of the C ABI.  Returns the status code."""
+    if not isinstance(desc_table, ctypes.Array):
+        desc_table = (fp8bq_desc * len(desc_table))(*desc_table)
+    n = len(desc_table) if n_tensors is None else n_tensors
+    return lib().fp8bq_quantize_batched(desc_table, n, _stream(stream))
+
+
+def fp8bq_status_string(status: int) -> str:
+    return lib().fp8bq_status_string(status).decode()
+
+
+def fp8bq_sync_status(stream=None) -> int:
+    return lib().fp8bq_sync_status(_stream(stream))
+
+
+def fp8bq_version() -> int:
+    return lib().fp8bq_version()
+
+
+def fp8bq_set_path(path: int) -> int:
+    return lib().fp8bq_set_path(path)
+
+
+def fp8bq_get_path() -> int:
+    return lib().fp8bq_get_path()
+
+
+def fp8bq_path_for(desc: fp8bq_desc) -> int:
+    return lib().fp8bq_path_for(ctypes.byref(desc))
+
+
+def fp8bq_debug_set_wait_limit_ns(ns: int) -> int:
+    return lib().fp8bq_debug_set_wait_limit_ns(ns)
+
+
+def fp8bq_debug_set_inject(flags: int) -> int:
+    return lib().fp8bq_debug_set_inject(flags)
+
+
+def check(status: int, what: str = "") -> None:
+    if status != FP8BQ_OK:
+        raise Fp8bqError(status, what)
+
+
+# ----------------------------------------------------------------- PyTorch conveniences
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FP8BQ_BF16
+    if t.dtype == torch.float32:
+        return FP8BQ_F32
+    raise TypeError(f"input must be bfloat16 or float32, got {t.dtype}")
+
+
+def make_desc(x, y, s, block=DEFAULT_BLOCK) -> fp8bq_desc:
+    """Descriptor for a CUDA tensor ``x`` of shape [M, N] or [E, M, N] (unit
+    stride along N), its e4m3fn output ``y`` (contiguous, same shape) and its
+    descale ``s`` (contiguous [(E,) ceil(M/bm), ceil(N/bn)])."""
+    if x.dim() not in (2, 3):
+        raise ValueError("expected a 2-D weight or a 3-D stack of expert weights")
+    if x.shape[-1] > 1 and x.stride(-1) != 1:
+        raise ValueError("the last dimension of the input must have unit stride")
+    d = fp8bq_desc()
+    d.x, d.y_u8, d.descale_f32 = _ptr(x), _ptr(y), _ptr(s)
+    d.M, d.N = int(x.shape[-2]), int(x.shape[-1])
+    d.ld = int(x.stride(-2)) if x.shape[-2] > 1 else max(int(x.shape[-1]), 1)
+    d.ld = max(d.ld, d.N)
+    d.batch = int(x.shape[0]) if x.dim() == 3 else 1
+    gm, gn = -(-d.M // block[0]), -(-d.N // block[1])
+    d.x_batch_stride = int(x.stride(0)) if x.dim() == 3 else 0
+    d.y_batch_stride = d.M * d.N if x.dim() == 3 else 0
+    d.s_batch_stride = gm * gn if x.dim() == 3 else 0
+    d.dtype_in = _dtype_code(x)
+    d.block_m, d.block_n = int(block[0]), int(block[1])
+    return d
+
+
+def _outputs(x, block):
+    import torch
+    M, N = x.shape[-2], x.shape[-1]
+    gm, gn = -(-M // block[0]), -(-N // block[1])
+    y = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty((*x.shape[:-2], gm, gn), dtype=torch.float32, device=x.device)
+    return y, s
+
+
+def scaled_fp8_blockwise(data_hp, weight_block_size=DEFAULT_BLOCK, stream=None):
+    """Quantize one bf16/fp32 CUDA weight ([M, N], or [E, M, N] for a stack of
+    experts) to e4m3fn with one fp32 descale per block.
+
+    Returns ``(fp8_data, descale)``: ``fp8_data`` has the input's shape and
+    dtype ``torch.float8_e4m3fn``; ``descale`` is [(E,) ceil(M/bm), ceil(N/bn)]
+    fp32 (the "weight_scale_inv" of the rollout engine).
+    """
+    block = tuple(int(b) for b in weight_block_size)
+    y, s = _outputs(data_hp, block)
+    check(fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream),
+          "scaled_fp8_blockwise")
+    return y, s
+
+
+def quant_weights(weights: Iterable, weight_block_size=DEFAULT_BLOCK, stream=None):
+    """Quantize every (name, tensor) pair in one grouped call and return the
+    list the rollout engine loads: (name, fp8 weight) followed by
+    (name + "_scale_inv", descale) for each input, in input order."""
+    block = tuple(int(b) for b in weight_block_size)
+    items, descs = [], []
+    for name, w in weights:
+        y, s = _outputs(w, block)
+        items.append((name, y, s, w))
+        descs.append(make_desc(w, y, s, block))
+    check(fp8bq_quantize_batched(descs, stream=stream), "quant_weights")
+    out = []
+    for name, y, s, _w in items:
+        out.append((name, y))
+        out.append((name + "_scale_inv", s))
+    return out

@@ -1,0 +1,63 @@
+"""Build the in-tree shared library ``libfp8bq.so`` for sm_100a with nvcc.
+
+    python -m blockwise_fp8_weight_b200.build [--verbose-ptxas]
+
+The library links the CUDA runtime statically, so it does not depend on
+which libcudart the host process (e.g. PyTorch) loaded.
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(PKG)
+CSRC = os.path.join(PKG, "csrc")
+SOURCES = [os.path.join(CSRC, f) for f in ("fp8bq_api.cu", "fp8bq_kernels.cu")]
+HEADERS = [os.path.join(CSRC, f) for f in ("fp8bq_internal.h", "fp8bq_device.cuh")] + [
+    os.path.join(ROOT, "include", "fp8bq.h")]
+LIB = os.path.join(PKG, "libfp8bq.so")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
+         "-cudart", "static", "--expt-relaxed-constexpr",
+         # IEEE division/sqrt and no flush-to-zero (nvcc's defaults, stated explicitly)
+         "-prec-div=true", "-prec-sqrt=true", "-ftz=false", "-fmad=true"]
+
+
+def nvcc() -> str:
+    for cand in (os.environ.get("NVCC"), shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found")
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False) -> str:
+    if not force and not verbose_ptxas and up_to_date():
+        return LIB
+    tmp = LIB + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *SOURCES]
+    if verbose_ptxas:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--verbose-ptxas", action="store_true")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    sys.exit(0)

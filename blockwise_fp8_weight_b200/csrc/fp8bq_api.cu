@@ -1,0 +1,471 @@
+// fp8bq_api.cu -- the C ABI of the blockwise FP8 weight quantizer: argument
+// checks, the choice of kernel variant per tensor, grouping into launches,
+// tensor-map encoding for the TMA variant, and status reporting.
+//
+// The entry points follow scaled_fp8_blockwise(data_hp, weight_block_size)
+// (verl docs "fp8_kernel.py -- FP8 量化内核", section 1 "统一入口") and the
+// per-layer quant_weights stream ("vllm_fp8_utils.py" docs, section 3
+// "权重量化").  The pages launch one kernel per tensor; here a whole list of
+// tensors becomes one persistent launch per kernel variant.
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
+
+#include <algorithm>
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/fp8bq.h"
+#include "fp8bq_internal.h"
+
+using namespace fp8bq;
+
+namespace {
+
+std::atomic<int> g_path{FP8BQ_PATH_AUTO};
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<uint32_t> g_inject{0};
+
+int esize_of(int32_t dtype) { return dtype == FP8BQ_BF16 ? 2 : 4; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+bool is_pow2(int64_t v) { return v > 0 && (v & (v - 1)) == 0; }
+
+// ------------------------------------------------------------------ checks
+
+fp8bq_status check_desc(const fp8bq_desc &D, bool *empty) {
+    if (D.dtype_in != FP8BQ_BF16 && D.dtype_in != FP8BQ_F32) return FP8BQ_ERR_DTYPE;
+    if (D.block_m < 1 || D.block_n < 1 || (int64_t)D.block_m * D.block_n > 65536)
+        return FP8BQ_ERR_BLOCK;
+    if (D.M < 0 || D.N < 0 || D.batch < 0 || D.ld < D.N || D.ld < 0) return FP8BQ_ERR_SHAPE;
+    if (D.M >= (1ll << 31) || D.N >= (1ll << 31)) return FP8BQ_ERR_SHAPE;
+    *empty = D.M == 0 || D.N == 0 || D.batch == 0;
+    if (*empty) return FP8BQ_OK;
+    if (D.batch > 1 && (D.x_batch_stride < 0 || D.y_batch_stride < 0 || D.s_batch_stride < 0))
+        return FP8BQ_ERR_SHAPE;
+    const int64_t tiles = D.batch * cdiv(D.M, D.block_m) * cdiv(D.N, D.block_n);
+    if (tiles >= (1ll << 31)) return FP8BQ_ERR_SHAPE;
+    if (D.x == nullptr || D.y_u8 == nullptr || D.descale_f32 == nullptr) return FP8BQ_ERR_NULL;
+    const int es = esize_of(D.dtype_in);
+    if (((uintptr_t)D.x % es) != 0 || ((uintptr_t)D.descale_f32 % 4) != 0) return FP8BQ_ERR_ALIGN;
+    if (D.batch > 1) {
+        const int64_t gm = cdiv(D.M, D.block_m), gn = cdiv(D.N, D.block_n);
+        if (D.y_batch_stride < D.M * D.N || D.s_batch_stride < gm * gn) return FP8BQ_ERR_OVERLAP;
+    }
+    return FP8BQ_OK;
+}
+
+struct Span {
+    uintptr_t lo, hi;  // [lo, hi)
+    bool out;
+};
+
+// Byte ranges each argument spans.  Outputs may overlap nothing; inputs may
+// overlap each other.
+fp8bq_status check_overlap(const fp8bq_desc *t, int n, const std::vector<char> &empty) {
+    std::vector<Span> sp;
+    sp.reserve((size_t)n * 3);
+    for (int i = 0; i < n; ++i) {
+        if (empty[i]) continue;
+        const fp8bq_desc &D = t[i];
+        const int64_t es = esize_of(D.dtype_in);
+        const int64_t b1 = D.batch - 1;
+        const int64_t gm = cdiv(D.M, D.block_m), gn = cdiv(D.N, D.block_n);
+        const int64_t xe = (b1 * (D.batch > 1 ? D.x_batch_stride : 0) + (D.M - 1) * D.ld + D.N) * es;
+        const int64_t ye = b1 * (D.batch > 1 ? D.y_batch_stride : 0) + D.M * D.N;
+        const int64_t se = (b1 * (D.batch > 1 ? D.s_batch_stride : 0) + gm * gn) * 4;
+        sp.push_back({(uintptr_t)D.x, (uintptr_t)D.x + (uintptr_t)xe, false});
+        sp.push_back({(uintptr_t)D.y_u8, (uintptr_t)D.y_u8 + (uintptr_t)ye, true});
+        sp.push_back({(uintptr_t)D.descale_f32, (uintptr_t)D.descale_f32 + (uintptr_t)se, true});
+    }
+    std::sort(sp.begin(), sp.end(), [](const Span &a, const Span &b) { return a.lo < b.lo; });
+    // Sweep: track the furthest end of any output and of any input seen so far.
+    uintptr_t out_end = 0, in_end = 0;
+    for (const Span &s : sp) {
+        if (s.out) {
+            if (s.lo < out_end || s.lo < in_end) return FP8BQ_ERR_OVERLAP;
+            out_end = std::max(out_end, s.hi);
+        } else {
+            if (s.lo < out_end) return FP8BQ_ERR_OVERLAP;
+            in_end = std::max(in_end, s.hi);
+        }
+    }
+    return FP8BQ_OK;
+}
+
+// ------------------------------------------------------------------ device
+
+fp8bq_status check_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return FP8BQ_ERR_DEVICE;
+    }
+    static std::atomic<int> ok_cache[64];  // 0 unknown, 1 ok, 2 not usable
+    if (dev < 64) {
+        const int c = ok_cache[dev].load();
+        if (c) return c == 1 ? FP8BQ_OK : FP8BQ_ERR_DEVICE;
+    }
+    int major = 0, minor = 0;
+    bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+              cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+              major == 10 && minor == 0;
+    if (!ok) cudaGetLastError();
+    if (dev < 64) ok_cache[dev].store(ok ? 1 : 2);
+    return ok ? FP8BQ_OK : FP8BQ_ERR_DEVICE;
+}
+
+// ------------------------------------------------------------------ variants
+
+bool vector_fits(const fp8bq_desc &D, Variant v) {
+    const int es = esize_of(D.dtype_in), vec = 16 / es;
+    const int team = kVecTeamThreads(v, es), slots = kVecSlots(v);
+    if (D.block_n % vec) return false;
+    const int vpr = D.block_n / vec;
+    if (!is_pow2(vpr) || vpr > team) return false;
+    return cdiv(D.block_m, team / vpr) <= slots;
+}
+
+// Alignment that lets whole 16-byte input vectors and whole output vectors
+// (vec bytes of e4m3 codes) be moved without straddling a row end.
+bool vector_aligned(const fp8bq_desc &D) {
+    const int es = esize_of(D.dtype_in), vec = 16 / es;
+    if ((uintptr_t)D.x % 16 || (D.ld * es) % 16 || D.N % vec) return false;
+    if ((uintptr_t)D.y_u8 % vec) return false;
+    if (D.batch > 1 && ((D.x_batch_stride * es) % 16 || D.y_batch_stride % vec)) return false;
+    return true;
+}
+
+Variant vector_variant(const fp8bq_desc &D) {
+    for (Variant v : {Variant::VecT16, Variant::VecT64, Variant::VecTBig})
+        if (vector_fits(D, v)) return v;
+    return Variant::Generic;
+}
+
+bool tma_fits(const fp8bq_desc &D) {
+    const int es = esize_of(D.dtype_in), vec = 16 / es;
+    if (D.block_m > 256 || D.block_n > 256 || (D.block_n * es) % 16) return false;
+    if ((int64_t)D.block_m * D.block_n * es > 128 * 128 * es) return false;
+    const int vpr = D.block_n / vec;
+    if (!is_pow2(vpr) || vpr > kTmaConsumerThreads) return false;
+    const int64_t slots = 128 * 128 * es / 16 / kTmaConsumerThreads;
+    if (cdiv(D.block_m, kTmaConsumerThreads / vpr) > slots) return false;
+    if (D.batch > 1 && D.x_batch_stride == 0) return false;
+    return vector_aligned(D);
+}
+
+Variant choose(const fp8bq_desc &D, int path) {
+    if (path == FP8BQ_PATH_GENERIC) return Variant::Generic;
+    if (path == FP8BQ_PATH_TMA && tma_fits(D)) return Variant::Tma;
+    if (!vector_aligned(D)) return Variant::Generic;
+    return vector_variant(D);
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+struct MapKey {
+    uintptr_t x;
+    int64_t M, N, ld, batch, xbs;
+    int32_t dtype, bm, bn;
+    bool operator==(const MapKey &o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapKeyHash {
+    size_t operator()(const MapKey &k) const {
+        const uint64_t *w = reinterpret_cast<const uint64_t *>(&k);
+        uint64_t h = 1469598103934665603ull;
+        for (size_t i = 0; i < sizeof(MapKey) / 8; ++i) h = (h ^ w[i]) * 1099511628211ull;
+        return (size_t)h;
+    }
+};
+
+// Encoded maps are cached by (pointer, shape, strides, block): a trainer's
+// weight buffers are the same on every sync step, so steady state encodes
+// nothing.
+bool encode_map(const fp8bq_desc &D, CUtensorMap *out) {
+    static std::mutex mu;
+    static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+    MapKey key;
+    std::memset(&key, 0, sizeof key);
+    key.x = (uintptr_t)D.x;
+    key.M = D.M;
+    key.N = D.N;
+    key.ld = D.ld;
+    key.batch = D.batch;
+    key.xbs = D.batch > 1 ? D.x_batch_stride : D.M * D.ld;
+    key.dtype = D.dtype_in;
+    key.bm = D.block_m;
+    key.bn = D.block_n;
+    {
+        std::lock_guard<std::mutex> g(mu);
+        auto it = cache.find(key);
+        if (it != cache.end()) {
+            *out = it->second;
+            return true;
+        }
+    }
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const int es = esize_of(D.dtype_in);
+    cuuint64_t dims[3] = {(cuuint64_t)D.N, (cuuint64_t)D.M, (cuuint64_t)D.batch};
+    cuuint64_t strides[2] = {(cuuint64_t)(D.ld * es), (cuuint64_t)(key.xbs * es)};
+    cuuint32_t box[3] = {(cuuint32_t)D.block_n, (cuuint32_t)D.block_m, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUtensorMap m;
+    CUresult r = fn(&m,
+                    D.dtype_in == FP8BQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                    3, const_cast<void *>(D.x), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> g(mu);
+    if (cache.size() > 8192) cache.clear();
+    cache.emplace(key, m);
+    *out = m;
+    return true;
+}
+
+// ------------------------------------------------------------------ launches
+
+void fill_tile_desc(const fp8bq_desc &D, uint32_t begin, TileDesc *o) {
+    o->x = D.x;
+    o->y = D.y_u8;
+    o->s = D.descale_f32;
+    o->ld = D.ld;
+    o->xbs = D.batch > 1 ? D.x_batch_stride : 0;
+    o->ybs = D.batch > 1 ? D.y_batch_stride : 0;
+    o->sbs = D.batch > 1 ? D.s_batch_stride : 0;
+    o->M = (int32_t)D.M;
+    o->N = (int32_t)D.N;
+    o->bm = D.block_m;
+    o->bn = D.block_n;
+    o->gm = (int32_t)cdiv(D.M, D.block_m);
+    o->gn = (int32_t)cdiv(D.N, D.block_n);
+    o->tile_begin = begin;
+    o->tiles = (uint32_t)(D.batch * o->gm * o->gn);
+}
+
+template <int MAXD>
+void pack_header(DescPack<MAXD> &p) {
+    p.n = 0;
+    p.total_tiles = 0;
+    p.inject = g_inject.load();
+    p.pad_ = 0;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+}
+
+// Launch one group (same variant, dtype and, for vector/TMA, block shape) in
+// chunks that fit the parameter pack and keep the tile count below 2^31.
+template <int MAXD>
+cudaError_t launch_group(Variant v, int es, const fp8bq_desc *t, const std::vector<int> &idx,
+                         cudaStream_t st) {
+    static thread_local DescPack<MAXD> p;  // large: keep it off the stack
+    size_t i = 0;
+    while (i < idx.size()) {
+        pack_header(p);
+        while (i < idx.size() && p.n < MAXD) {
+            const fp8bq_desc &D = t[idx[i]];
+            const uint64_t tiles = (uint64_t)D.batch * cdiv(D.M, D.block_m) * cdiv(D.N, D.block_n);
+            if (p.n > 0 && (uint64_t)p.total_tiles + tiles >= (1ull << 31)) break;
+            fill_tile_desc(D, p.total_tiles, &p.d[p.n]);
+            p.total_tiles += (uint32_t)tiles;
+            ++p.n;
+            ++i;
+        }
+        const cudaError_t e = v == Variant::Generic ? launch_generic<MAXD>(es, p, st)
+                                                    : launch_vector<MAXD>(v, es, p, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int> &idx,
+                             const std::vector<CUtensorMap> &maps, cudaStream_t st) {
+    static thread_local TmaPack<kMaxDescTma> P;
+    size_t i = 0;
+    while (i < idx.size()) {
+        pack_header(P.p);
+        while (i < idx.size() && P.p.n < kMaxDescTma) {
+            const fp8bq_desc &D = t[idx[i]];
+            const uint64_t tiles = (uint64_t)D.batch * cdiv(D.M, D.block_m) * cdiv(D.N, D.block_n);
+            if (P.p.n > 0 && (uint64_t)P.p.total_tiles + tiles >= (1ull << 31)) break;
+            fill_tile_desc(D, P.p.total_tiles, &P.p.d[P.p.n]);
+            P.maps[P.p.n] = maps[i];
+            P.p.total_tiles += (uint32_t)tiles;
+            ++P.p.n;
+            ++i;
+        }
+        const cudaError_t e = launch_tma(es, P, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+struct GroupKey {
+    Variant v;
+    int es, bm, bn;
+    bool operator==(const GroupKey &o) const {
+        return v == o.v && es == o.es && bm == o.bm && bn == o.bn;
+    }
+};
+
+fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
+    if (n < 0) return FP8BQ_ERR_ARG;
+    if (n > 0 && table == nullptr) return FP8BQ_ERR_NULL;
+    std::vector<char> empty((size_t)n, 0);
+    bool any = false;
+    for (int i = 0; i < n; ++i) {
+        bool e = false;
+        const fp8bq_status s = check_desc(table[i], &e);
+        if (s != FP8BQ_OK) return s;
+        empty[i] = e;
+        any |= !e;
+    }
+    if (!any) return FP8BQ_OK;
+    const fp8bq_status so = check_overlap(table, n, empty);
+    if (so != FP8BQ_OK) return so;
+    const fp8bq_status sd = check_device();
+    if (sd != FP8BQ_OK) return sd;
+
+    // Group tensors by kernel variant, keeping the caller's order inside a group.
+    const int path = g_path.load();
+    std::vector<GroupKey> keys;
+    std::vector<std::vector<int>> members;
+    std::vector<std::vector<CUtensorMap>> maps;
+    for (int i = 0; i < n; ++i) {
+        if (empty[i]) continue;
+        const fp8bq_desc &D = table[i];
+        Variant v = choose(D, path);
+        CUtensorMap m;
+        if (v == Variant::Tma && !encode_map(D, &m)) v = choose(D, FP8BQ_PATH_VECTOR);
+        GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? 0 : D.block_m,
+                   v == Variant::Generic ? 0 : D.block_n};
+        size_t g = 0;
+        while (g < keys.size() && !(keys[g] == k)) ++g;
+        if (g == keys.size()) {
+            keys.push_back(k);
+            members.emplace_back();
+            maps.emplace_back();
+        }
+        members[g].push_back(i);
+        if (v == Variant::Tma) maps[g].push_back(m);
+    }
+    for (size_t g = 0; g < keys.size(); ++g) {
+        cudaError_t e;
+        if (keys[g].v == Variant::Tma)
+            e = launch_tma_group(keys[g].es, table, members[g], maps[g], stream);
+        else if (members[g].size() <= (size_t)kMaxDescSmall)
+            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, table, members[g], stream);
+        else
+            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, table, members[g], stream);
+        if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
+    }
+    return FP8BQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8bq_status fp8bq_quantize(const void *x, fp8bq_dtype dtype_in, int64_t M, int64_t N, int64_t ld,
+                            int block_m, int block_n, uint8_t *y_u8, float *descale_f32,
+                            cudaStream_t stream) {
+    fp8bq_desc D;
+    std::memset(&D, 0, sizeof D);
+    D.x = x;
+    D.y_u8 = y_u8;
+    D.descale_f32 = descale_f32;
+    D.M = M;
+    D.N = N;
+    D.ld = ld;
+    D.batch = 1;
+    D.dtype_in = (int32_t)dtype_in;
+    D.block_m = block_m;
+    D.block_n = block_n;
+    return run(&D, 1, stream);
+}
+
+fp8bq_status fp8bq_quantize_batched(const fp8bq_desc *desc_table, int n_tensors,
+                                    cudaStream_t stream) {
+    return run(desc_table, n_tensors, stream);
+}
+
+const char *fp8bq_status_string(fp8bq_status s) {
+    switch (s) {
+        case FP8BQ_OK: return "FP8BQ_OK";
+        case FP8BQ_ERR_NULL: return "FP8BQ_ERR_NULL: a required pointer is NULL";
+        case FP8BQ_ERR_SHAPE: return "FP8BQ_ERR_SHAPE: invalid shape, stride or batch";
+        case FP8BQ_ERR_BLOCK: return "FP8BQ_ERR_BLOCK: invalid block shape";
+        case FP8BQ_ERR_DTYPE: return "FP8BQ_ERR_DTYPE: unknown input dtype";
+        case FP8BQ_ERR_OVERLAP: return "FP8BQ_ERR_OVERLAP: an output overlaps an input or output";
+        case FP8BQ_ERR_DEVICE: return "FP8BQ_ERR_DEVICE: no usable sm_100 device or CUDA error";
+        case FP8BQ_ERR_DEVICE_TIMEOUT:
+            return "FP8BQ_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
+        case FP8BQ_ERR_ALIGN: return "FP8BQ_ERR_ALIGN: misaligned input or descale pointer";
+        case FP8BQ_ERR_ARG: return "FP8BQ_ERR_ARG: invalid argument";
+    }
+    return "FP8BQ_?: unknown status";
+}
+
+fp8bq_status fp8bq_sync_status(cudaStream_t stream) {
+    if (check_device() != FP8BQ_OK) return FP8BQ_ERR_DEVICE;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8BQ_ERR_DEVICE;
+    }
+    uint32_t w = 0;
+    if (read_and_clear_error_word(&w) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8BQ_ERR_DEVICE;
+    }
+    return w ? FP8BQ_ERR_DEVICE_TIMEOUT : FP8BQ_OK;
+}
+
+int fp8bq_version(void) { return FP8BQ_VERSION; }
+
+fp8bq_status fp8bq_set_path(fp8bq_path path) {
+    if (path < FP8BQ_PATH_AUTO || path > FP8BQ_PATH_GENERIC) return FP8BQ_ERR_ARG;
+    g_path.store((int)path);
+    return FP8BQ_OK;
+}
+
+fp8bq_path fp8bq_get_path(void) { return (fp8bq_path)g_path.load(); }
+
+int fp8bq_path_for(const fp8bq_desc *desc) {
+    if (desc == nullptr) return -1;
+    bool e = false;
+    if (check_desc(*desc, &e) != FP8BQ_OK) return -1;
+    switch (choose(*desc, g_path.load())) {
+        case Variant::Tma: return FP8BQ_PATH_TMA;
+        case Variant::Generic: return FP8BQ_PATH_GENERIC;
+        default: return FP8BQ_PATH_VECTOR;
+    }
+}
+
+fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns) {
+    g_wait_limit_ns.store(ns ? ns : 2000000000ull);
+    return FP8BQ_OK;
+}
+
+fp8bq_status fp8bq_debug_set_inject(uint32_t flags) {
+    if (flags & ~FP8BQ_INJECT_DROP_FIRST_LOAD) return FP8BQ_ERR_ARG;
+    g_inject.store(flags);
+    return FP8BQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+// fp8bq_internal.h -- what the host side of the library and its kernels share.
+#pragma once
+
+#include <cuda.h>  // CUtensorMap (type only; the driver entry point is fetched at run time)
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fp8bq {
+
+// The eps floor of the block absmax.  The pages print the floor (absmax =
+// max(max|x|, eps)) but not its value; 1e-10 is this library's reading.
+constexpr float kEps = 1e-10f;
+// Largest finite float8_e4m3fn value: the fp8_max / -fp8_min of the scale step.
+constexpr float kFp8Max = 448.0f;
+
+// One weight tensor as the kernels see it (kernel-parameter space).
+struct TileDesc {
+    const void *x;      // input base
+    uint8_t *y;         // e4m3fn output base
+    float *s;           // descale base
+    int64_t ld;         // input row stride, elements
+    int64_t xbs;        // input batch stride, elements
+    int64_t ybs;        // output batch stride, bytes
+    int64_t sbs;        // descale batch stride, floats
+    int32_t M, N;       // matrix shape
+    int32_t bm, bn;     // block shape
+    int32_t gm, gn;     // block grid of one matrix
+    uint32_t tile_begin;// first tile id of this tensor within the launch
+    uint32_t tiles;     // batch * gm * gn
+};
+static_assert(sizeof(TileDesc) == 88, "TileDesc layout");
+
+// Grouped-launch parameters.  MAXD bounds the descriptors per launch so the
+// whole pack stays inside the 32 KB kernel-parameter limit.
+template <int MAXD>
+struct DescPack {
+    int32_t n;              // descriptors used
+    uint32_t total_tiles;   // sum of tiles
+    uint32_t inject;        // FP8BQ_INJECT_* flags (TMA kernel)
+    uint32_t pad_;
+    uint64_t wait_limit_ns; // bound of every device wait (TMA kernel)
+    TileDesc d[MAXD];
+};
+
+template <int MAXD>
+struct alignas(64) TmaPack {
+    CUtensorMap maps[MAXD];  // one 3-D map per descriptor: {N, M, batch}, box {bn, bm, 1}
+    DescPack<MAXD> p;
+};
+
+constexpr int kMaxDescSmall = 8;
+constexpr int kMaxDescLarge = 320;  // 320 * 88 B + header = 28.2 KB
+constexpr int kMaxDescTma = 128;    // 128 * (128 + 88) B + header = 27.7 KB
+static_assert(sizeof(DescPack<kMaxDescLarge>) < 32000, "kernel parameter limit");
+static_assert(sizeof(TmaPack<kMaxDescTma>) < 32000, "kernel parameter limit");
+
+// Kernel variants, by input element size and team shape.
+enum class Variant : int {
+    Generic = 0,
+    VecT16 = 1,   // a team of 16 threads per block (blocks of <= 16 vectors)
+    VecT64 = 2,   // a team of 64 threads per block (<= 512 vectors)
+    VecTBig = 3,  // one team per CTA (<= 2048 vectors)
+    Tma = 4,
+};
+
+// Launchers (fp8bq_kernels.cu).  Each returns cudaSuccess or the launch error.
+template <int MAXD>
+cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st);
+template <int MAXD>
+cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
+cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st);
+
+// Device error word access (fp8bq_kernels.cu).
+cudaError_t read_and_clear_error_word(uint32_t *out);
+
+// Team geometry used by the vector kernels (host eligibility must agree).
+constexpr int kVecTeamThreads(Variant v, int esize) {
+    return v == Variant::VecT16 ? 16 : v == Variant::VecT64 ? 64 : (esize == 2 ? 256 : 512);
+}
+constexpr int kVecSlots(Variant v) { return v == Variant::VecT16 ? 1 : 8; }
+
+constexpr int kTmaConsumerThreads = 256;
+constexpr int kTmaStageBytes = 32768;
+
+}  // namespace fp8bq

@@ -1,0 +1,502 @@
+// fp8bq_kernels.cu -- sm_100a kernels of the blockwise FP8 weight quantizer.
+//
+// Every kernel computes, for each [bm, bn] block of each tensor of a grouped
+// launch (verl docs "fp8_kernel.py -- FP8 量化内核", section 2 "Triton 实现"):
+//   a = max(max |x| over the block's valid elements, eps)
+//   s = a / 448, r = 1 / s                (IEEE fp32 divisions)
+//   y = e4m3fn(clamp(x * r, -448, 448))   (single-rounded multiply, RNE, satfinite)
+//   descale = s
+// The block absmax is taken on bit patterns: for a non-negative IEEE value the
+// unsigned integer order of the bits equals the numeric order, so max over
+// (bits & 0x7fff...) is exactly the fp32 absmax (bf16 is the top half of fp32).
+//
+// The pages' kernel runs one Triton program per block on a 2-D grid per tensor
+// and one launch per tensor.  Here one persistent launch walks the tiles of
+// all tensors of a group (the descriptor table travels in the kernel
+// parameters); three variants share the arithmetic:
+//   k_vector   16-byte coalesced global loads into registers, next tile
+//              prefetched while the current one is reduced and stored;
+//   k_tma      a producer warp streams 2-D TMA tiles into a shared-memory
+//              ring, consumer warps reduce and quantize (bounded waits);
+//   k_generic  element-wise loads, one warp per block: any alignment,
+//              stride or block shape.
+#include "fp8bq_device.cuh"
+#include "fp8bq_internal.h"
+
+namespace fp8bq {
+
+// Bit 0: a consumer or producer wait ran out.  Bit 1: the end-of-kernel drain
+// of in-flight TMA copies ran out.
+__device__ uint32_t g_error_word;
+
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
+
+// Tile geometry shared by all kernels.
+struct Tile {
+    const char *src;  // first element of the block
+    uint8_t *dst;     // first output byte of the block
+    float *sdst;      // descale slot
+    int64_t ld;       // input row stride, elements
+    int64_t ldy;      // output row stride (= N)
+    int rows, cols;   // valid extent
+    int b, bi, bj;    // coordinates (TMA)
+};
+
+template <int ESIZE, int MAXD>
+__device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d) {
+    while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
+    const TileDesc &D = p.d[d];
+    const uint32_t local = t - D.tile_begin;
+    const uint32_t per = (uint32_t)D.gm * (uint32_t)D.gn;
+    const uint32_t b = local / per;
+    const uint32_t rem = local - b * per;
+    const uint32_t bi = rem / (uint32_t)D.gn;
+    const uint32_t bj = rem - bi * (uint32_t)D.gn;
+    const int64_t r0 = (int64_t)bi * D.bm, c0 = (int64_t)bj * D.bn;
+    Tile T;
+    T.src = (const char *)D.x + ((int64_t)b * D.xbs + r0 * D.ld + c0) * ESIZE;
+    T.dst = D.y + (int64_t)b * D.ybs + r0 * D.N + c0;
+    T.sdst = D.s + (int64_t)b * D.sbs + (int64_t)bi * D.gn + bj;
+    T.ld = D.ld;
+    T.ldy = D.N;
+    T.rows = (int)min((int64_t)D.bm, (int64_t)D.M - r0);
+    T.cols = (int)min((int64_t)D.bn, (int64_t)D.N - c0);
+    T.b = (int)b;
+    T.bi = (int)bi;
+    T.bj = (int)bj;
+    return T;
+}
+
+// absmax bits of a 16-byte vector
+template <int ESIZE>
+__device__ __forceinline__ uint32_t vec_absmax(const uint4 &v, uint32_t m) {
+    if constexpr (ESIZE == 2) {
+        m = __vmaxu2(m, v.x & 0x7fff7fffu);
+        m = __vmaxu2(m, v.y & 0x7fff7fffu);
+        m = __vmaxu2(m, v.z & 0x7fff7fffu);
+        m = __vmaxu2(m, v.w & 0x7fff7fffu);
+    } else {
+        m = max(m, v.x & 0x7fffffffu);
+        m = max(m, v.y & 0x7fffffffu);
+        m = max(m, v.z & 0x7fffffffu);
+        m = max(m, v.w & 0x7fffffffu);
+    }
+    return m;
+}
+
+// fp32 bit pattern of the absmax accumulated by vec_absmax
+template <int ESIZE>
+__device__ __forceinline__ uint32_t absmax_to_f32_bits(uint32_t m) {
+    if constexpr (ESIZE == 2)
+        return max(m & 0xffffu, m >> 16) << 16;
+    else
+        return m;
+}
+
+// Quantize one 16-byte vector and store its codes (8 bytes for bf16, 4 for fp32).
+template <int ESIZE>
+__device__ __forceinline__ void vec_quant_store(const uint4 &v, float r, uint8_t *dst) {
+    if constexpr (ESIZE == 2) {
+        uint2 o;
+        o.x = dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.x), r),
+                              dev::scale_clamp(dev::bf16_hi(v.x), r)) |
+              (dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.y), r),
+                               dev::scale_clamp(dev::bf16_hi(v.y), r))
+               << 16);
+        o.y = dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.z), r),
+                              dev::scale_clamp(dev::bf16_hi(v.z), r)) |
+              (dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.w), r),
+                               dev::scale_clamp(dev::bf16_hi(v.w), r))
+               << 16);
+        dev::stg_stream_v2(dst, o);
+    } else {
+        uint32_t o = dev::cvt_e4m3x2(dev::scale_clamp(__uint_as_float(v.x), r),
+                                     dev::scale_clamp(__uint_as_float(v.y), r)) |
+                     (dev::cvt_e4m3x2(dev::scale_clamp(__uint_as_float(v.z), r),
+                                      dev::scale_clamp(__uint_as_float(v.w), r))
+                      << 16);
+        dev::stg_stream_u32(dst, o);
+    }
+}
+
+// ============================================================== vector kernel
+//
+// A team of TEAM threads owns one block at a time; a block of bm x bn
+// elements is bm rows of vpr = bn / VEC 16-byte vectors.  Thread `lane` of the
+// team holds the vectors (row0 + i * rstep, cv), i < V, with cv = lane % vpr,
+// row0 = lane / vpr, rstep = TEAM / vpr: consecutive lanes read consecutive
+// 16-byte pieces of a row, so each warp load covers whole 256-byte row
+// segments.  bm and bn are the same for every tensor of a launch.
+
+template <int ESIZE, int TEAM, int V, int CTA, int MAXD>
+__global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
+    k_vector(const __grid_constant__ DescPack<MAXD> p) {
+    constexpr int VEC = 16 / ESIZE;
+    constexpr int TEAMS = CTA / TEAM;
+    constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
+    __shared__ uint32_t red[2][TEAMS][WPT];
+
+    const int team = threadIdx.x / TEAM;
+    const int lane = threadIdx.x % TEAM;
+    const uint32_t stride = gridDim.x * TEAMS;
+    uint32_t t = blockIdx.x * TEAMS + team;
+    if (t >= p.total_tiles) return;
+
+    const int vpr = p.d[0].bn / VEC;  // power of two, <= TEAM (host-checked)
+    const int cv = lane & (vpr - 1);
+    const int row0 = lane / vpr;
+    const int rstep = TEAM / vpr;
+    const int colv = cv * VEC;
+    const uint32_t shfl_mask =
+        TEAM >= 32 ? 0xffffffffu : (((1u << TEAM) - 1u) << ((threadIdx.x & 31) & ~(TEAM - 1)));
+
+    auto load = [&](uint4 (&R)[V], const Tile &T) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int r = row0 + i * rstep;
+            if (r < T.rows && colv < T.cols)
+                R[i] = dev::ldg_stream_v4(T.src + ((int64_t)r * T.ld + colv) * ESIZE);
+            else
+                R[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+
+    auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) m = vec_absmax<ESIZE>(R[i], m);
+        m = absmax_to_f32_bits<ESIZE>(m);
+        if constexpr (TEAM <= 32) {
+#pragma unroll
+            for (int o = TEAM / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(shfl_mask, m, o));
+        } else {
+            m = __reduce_max_sync(0xffffffffu, m);
+            if ((lane & 31) == 0) red[it & 1][team][lane >> 5] = m;
+            dev::named_bar_sync(1 + team, TEAM);
+            m = red[it & 1][team][0];
+#pragma unroll
+            for (int w = 1; w < WPT; ++w) m = max(m, red[it & 1][team][w]);
+        }
+        float s, r;
+        dev::block_scale(m, kEps, s, r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int rr = row0 + i * rstep;
+            if (rr < T.rows && colv < T.cols)
+                vec_quant_store<ESIZE>(R[i], r, T.dst + (int64_t)rr * T.ldy + colv);
+        }
+        if (lane == 0) *T.sdst = s;
+    };
+
+    int d = 0;
+    uint4 A[V], B[V];
+    Tile ta = make_tile<ESIZE>(p, t, d);
+    load(A, ta);
+    uint32_t it = 0;
+    while (true) {
+        const uint32_t t1 = t + stride;
+        const bool h1 = t1 < p.total_tiles;
+        Tile tb;
+        if (h1) {
+            tb = make_tile<ESIZE>(p, t1, d);
+            load(B, tb);
+        }
+        process(A, ta, it++);
+        if (!h1) break;
+        const uint32_t t2 = t1 + stride;
+        const bool h2 = t2 < p.total_tiles;
+        if (h2) {
+            ta = make_tile<ESIZE>(p, t2, d);
+            load(A, ta);
+        }
+        process(B, tb, it++);
+        if (!h2) break;
+        t = t2;
+    }
+}
+
+// ============================================================== generic kernel
+//
+// One warp per block, element-wise loads and byte stores: any row stride,
+// alignment and block shape.  Two passes over the block (absmax, then
+// quantize); the second pass reads the block again, mostly from L1/L2.
+
+template <int ESIZE>
+__device__ __forceinline__ uint32_t elem_abs_bits(const char *p) {
+    if constexpr (ESIZE == 2)
+        return ((uint32_t)__ldg((const unsigned short *)p) & 0x7fffu) << 16;
+    else
+        return __float_as_uint(__ldg((const float *)p)) & 0x7fffffffu;
+}
+
+template <int ESIZE>
+__device__ __forceinline__ float elem_f32(const char *p) {
+    if constexpr (ESIZE == 2)
+        return __uint_as_float((uint32_t)__ldg((const unsigned short *)p) << 16);
+    else
+        return __ldg((const float *)p);
+}
+
+template <int ESIZE, int MAXD>
+__global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPack<MAXD> p) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t stride = gridDim.x * 8;
+    int d = 0;
+    for (uint32_t t = blockIdx.x * 8 + (threadIdx.x >> 5); t < p.total_tiles; t += stride) {
+        const Tile T = make_tile<ESIZE>(p, t, d);
+        uint32_t m = 0;
+        for (int r = 0; r < T.rows; ++r) {
+            const char *row = T.src + (int64_t)r * T.ld * ESIZE;
+            for (int c = lane; c < T.cols; c += 32) m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
+        }
+        m = __reduce_max_sync(0xffffffffu, m);
+        float s, rc;
+        dev::block_scale(m, kEps, s, rc);
+        for (int r = 0; r < T.rows; ++r) {
+            const char *row = T.src + (int64_t)r * T.ld * ESIZE;
+            uint8_t *out = T.dst + (int64_t)r * T.ldy;
+            for (int c = lane; c < T.cols; c += 32) {
+                const float v = dev::scale_clamp(elem_f32<ESIZE>(row + c * ESIZE), rc);
+                out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
+            }
+        }
+        if (lane == 0) *T.sdst = s;
+    }
+}
+
+// ============================================================== TMA kernel
+//
+// Warp 0 (one elected lane) is the producer: for each tile of this CTA it
+// waits until the ring slot is free, arms the slot's "full" barrier with the
+// tile's byte count and issues one 3-D tensor-map load (no multicast).  Warps
+// 1..8 are consumers: they wait for "full", copy the tile from shared memory
+// into registers, release the slot ("empty"), reduce the absmax across the 8
+// warps, and quantize + store from registers.  Every wait is bounded; a wait
+// that runs out sets the device error word, all consumers leave together
+// (the reduction barrier also ORs a failure flag), and the producer waits
+// (bounded) for each copy it issued before it returns.
+
+template <int ESIZE, int STAGES>
+__global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
+    k_tma(const __grid_constant__ TmaPack<kMaxDescTma> P) {
+    constexpr int VEC = 16 / ESIZE;
+    constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
+    constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
+    extern __shared__ __align__(1024) uint8_t ring[];
+    __shared__ __align__(8) uint64_t full[STAGES];
+    __shared__ __align__(8) uint64_t empty[STAGES];
+    __shared__ uint32_t red[2][kTmaConsumerThreads / 32];
+    __shared__ volatile int abort_flag;
+
+    const DescPack<kMaxDescTma> &p = P.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            dev::mbar_init(&full[s], 1);
+            dev::mbar_init(&empty[s], kTmaConsumerThreads / 32);
+        }
+        abort_flag = 0;
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+
+    const int bm = p.d[0].bm, bn = p.d[0].bn;
+    const uint32_t tile_bytes = (uint32_t)(bm * bn * ESIZE);
+
+    if (warp == 0) {
+        if (lane != 0) return;
+        int d = 0;
+        uint32_t k = 0;
+        bool dropped0 = false;
+        for (uint32_t t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++k) {
+            const int st = (int)(k % STAGES);
+            const uint32_t round = k / STAGES;
+            if (round > 0 &&
+                !dev::mbar_wait_bounded(&empty[st], (round - 1) & 1u, p.wait_limit_ns, &abort_flag)) {
+                if (!abort_flag) {
+                    atomicOr(&g_error_word, 1u);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            const Tile T = make_tile<ESIZE>(p, t, d);
+            dev::mbar_arrive_expect_tx(&full[st], tile_bytes);
+            if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
+                dropped0 = true;  // fault injection: this slot's barrier can never complete
+            else
+                dev::tma_load_3d(ring + (size_t)st * STAGE_BYTES, &P.maps[d], &full[st],
+                                 T.bj * bn, T.bi * bm, T.b);
+        }
+        // Drain: each slot's last issued copy must land before the CTA exits.
+        const uint32_t issued = k;
+        for (int st = 0; st < STAGES && (uint32_t)st < issued; ++st) {
+            const uint32_t fills = (issued - (uint32_t)st + STAGES - 1) / STAGES;
+            if (dropped0 && st == 0 && fills == 1) continue;
+            if (!dev::mbar_wait_bounded(&full[st], (fills - 1) & 1u, kDrainLimitNs, nullptr))
+                atomicOr(&g_error_word, 2u);
+        }
+        return;
+    }
+
+    // consumers
+    const int ct = threadIdx.x - 32;
+    const int cw = ct >> 5;
+    const int vpr = bn / VEC;
+    const int cv = ct & (vpr - 1);
+    const int row0 = ct / vpr;
+    const int rstep = kTmaConsumerThreads / vpr;
+    const int colv = cv * VEC;
+    int d = 0;
+    uint32_t k = 0;
+    for (uint32_t t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++k) {
+        const int st = (int)(k % STAGES);
+        const bool ok = dev::mbar_wait_bounded(&full[st], (k / STAGES) & 1u, p.wait_limit_ns,
+                                               &abort_flag);
+        const Tile T = make_tile<ESIZE>(p, t, d);
+        uint4 R[V];
+        const uint8_t *stage = ring + (size_t)st * STAGE_BYTES;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int r = row0 + i * rstep;
+            if (ok && r < bm)
+                R[i] = *reinterpret_cast<const uint4 *>(stage + ((size_t)r * bn + colv) * ESIZE);
+            else
+                R[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        if (lane == 0 && ok) dev::mbar_arrive(&empty[st]);
+
+        uint32_t m = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) m = vec_absmax<ESIZE>(R[i], m);
+        m = __reduce_max_sync(0xffffffffu, absmax_to_f32_bits<ESIZE>(m));
+        if (lane == 0) red[k & 1][cw] = m;
+        if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
+            if (ct == 0) {
+                atomicOr(&g_error_word, 1u);
+                abort_flag = 1;
+            }
+            break;
+        }
+        m = red[k & 1][0];
+#pragma unroll
+        for (int w = 1; w < kTmaConsumerThreads / 32; ++w) m = max(m, red[k & 1][w]);
+        float s, r;
+        dev::block_scale(m, kEps, s, r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int rr = row0 + i * rstep;
+            if (rr < T.rows && colv < T.cols)
+                vec_quant_store<ESIZE>(R[i], r, T.dst + (int64_t)rr * T.ldy + colv);
+        }
+        if (ct == 0) *T.sdst = s;
+    }
+}
+
+// ============================================================== launchers
+
+namespace {
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <typename K>
+int resident_ctas(K kernel, int threads, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+        n < 1)
+        n = 1;
+    return n;
+}
+
+unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {
+    const uint64_t need = (work_units + (uint32_t)units_per_cta - 1) / (uint32_t)units_per_cta;
+    const uint64_t cap = (uint64_t)sm_count() * (uint64_t)ctas_per_sm;
+    return (unsigned)(need < cap ? (need ? need : 1) : cap);
+}
+
+template <int ESIZE, int TEAM, int V, int CTA, int MAXD>
+cudaError_t launch_vector_t(const DescPack<MAXD> &p, cudaStream_t st) {
+    auto kern = k_vector<ESIZE, TEAM, V, CTA, MAXD>;
+    static int occ = resident_ctas(kern, CTA, 0);
+    const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
+    kern<<<grid, CTA, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+template <int MAXD>
+cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st) {
+    if (esize == 2) {
+        switch (v) {
+            case Variant::VecT16: return launch_vector_t<2, 16, 1, 256, MAXD>(p, st);
+            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, MAXD>(p, st);
+            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, MAXD>(p, st);
+            default: return cudaErrorInvalidValue;
+        }
+    }
+    switch (v) {
+        case Variant::VecT16: return launch_vector_t<4, 16, 1, 256, MAXD>(p, st);
+        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, MAXD>(p, st);
+        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, MAXD>(p, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <int MAXD>
+cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) {
+    if (esize == 2) {
+        static int occ = resident_ctas(k_generic<2, MAXD>, 256, 0);
+        k_generic<2, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+    } else {
+        static int occ = resident_ctas(k_generic<4, MAXD>, 256, 0);
+        k_generic<4, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+namespace {
+template <int ESIZE, int STAGES>
+cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
+    constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
+    auto kern = k_tma<ESIZE, STAGES>;
+    static cudaError_t attr =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
+    kern<<<grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
+    return esize == 2 ? launch_tma_t<2, 6>(p, st) : launch_tma_t<4, 3>(p, st);
+}
+
+cudaError_t read_and_clear_error_word(uint32_t *out) {
+    uint32_t zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(out, g_error_word, sizeof(uint32_t));
+    if (e != cudaSuccess) return e;
+    if (*out) e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(uint32_t));
+    return e;
+}
+
+template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, const DescPack<kMaxDescSmall> &,
+                                                  cudaStream_t);
+template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, const DescPack<kMaxDescLarge> &,
+                                                  cudaStream_t);
+template cudaError_t launch_generic<kMaxDescSmall>(int, const DescPack<kMaxDescSmall> &,
+                                                   cudaStream_t);
+template cudaError_t launch_generic<kMaxDescLarge>(int, const DescPack<kMaxDescLarge> &,
+                                                   cudaStream_t);
+
+}  // namespace fp8bq

@@ -1,0 +1,199 @@
+/*
+ * fp8bq.h -- blockwise FP8 (float8_e4m3fn) weight quantizer for NVIDIA B200
+ * (sm_100a).  C ABI.
+ *
+ * The operation (verl documentation page "fp8_kernel.py -- FP8 量化内核",
+ * section 1 "统一入口" and section 2 "Triton 实现"): a high-precision [M, N]
+ * matrix is cut into [block_m, block_n] blocks (edge blocks are clipped to the
+ * matrix).  For each block
+ *
+ *     a        = max(max |x| over the block's valid elements, eps)
+ *     s        = a / 448                      (IEEE fp32 division)
+ *     r        = 1 / s                        (IEEE fp32 division)
+ *     y[i, j]  = e4m3fn(clamp(x[i, j] * r, -448, 448))
+ *     descale  = s
+ *
+ * where e4m3fn() rounds to nearest, ties to even, saturating, and keeps the
+ * sign of a result that rounds to zero; eps = 1e-10f.  The pages print the
+ * eps floor but not its value; 1e-10f is this library's reading.  The result
+ * is unique bit for bit: there is no summation, and max is order independent.
+ *
+ * The descale is the dequantization multiplier, x ~= decode(y) * descale,
+ * which the rollout engine loads as "<weight name>_scale_inv" ("vllm_fp8_utils.py"
+ * docs, section 3 "权重量化"; verl PR #4415 review, where it is a 2-D tensor
+ * after squeeze(-1)).
+ *
+ * Layouts (all row-major):
+ *   x        [M, N] bf16 or fp32 elements, row stride ld >= N (elements).
+ *   y        [M, N] bytes (e4m3fn bit patterns), contiguous (row stride N).
+ *   descale  [ceil(M/block_m), ceil(N/block_n)] fp32, contiguous.
+ *
+ * Ownership: the caller allocates and owns x, y and descale (device memory of
+ * the current device).  The library writes only y and descale, allocates no
+ * device memory per call, and keeps no pointer after a call returns.
+ *
+ * Execution: calls are asynchronous on `stream`, like a kernel launch.  All
+ * arguments are checked before anything is launched; a call that returns an
+ * error launched nothing.  Inputs must not overlap outputs, and outputs must
+ * not overlap each other (checked on the address ranges each argument spans).
+ * NaN and infinite inputs are outside the contract (no error, unspecified
+ * codes).
+ */
+#ifndef FP8BQ_H
+#define FP8BQ_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FP8BQ_API __attribute__((visibility("default")))
+#else
+#define FP8BQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FP8BQ_VERSION 10000 /* 1.0.0 */
+
+typedef enum fp8bq_dtype {
+    FP8BQ_BF16 = 0, /* bfloat16 input */
+    FP8BQ_F32 = 1   /* float32 input */
+} fp8bq_dtype;
+
+typedef enum fp8bq_status {
+    FP8BQ_OK = 0,
+    FP8BQ_ERR_NULL = 1,           /* a required pointer is NULL */
+    FP8BQ_ERR_SHAPE = 2,          /* M, N, batch or a stride negative; ld < N; M or N >= 2^31;
+                                     too many blocks in one tensor (>= 2^31) */
+    FP8BQ_ERR_BLOCK = 3,          /* block_m or block_n < 1, or block_m * block_n > 65536 */
+    FP8BQ_ERR_DTYPE = 4,          /* dtype_in not an fp8bq_dtype */
+    FP8BQ_ERR_OVERLAP = 5,        /* an output overlaps an input or another output */
+    FP8BQ_ERR_DEVICE = 6,         /* no usable CUDA device, device is not sm_100, or a CUDA
+                                     call failed */
+    FP8BQ_ERR_DEVICE_TIMEOUT = 7, /* a bounded wait inside a kernel ran out (reported by
+                                     fp8bq_sync_status) */
+    FP8BQ_ERR_ALIGN = 8,          /* x not aligned to its element size, or descale not 4-byte
+                                     aligned */
+    FP8BQ_ERR_ARG = 9             /* other invalid argument (n_tensors < 0, unknown path) */
+} fp8bq_status;
+
+/*
+ * Quantize one matrix: scaled_fp8_blockwise(data_hp, weight_block_size) of the
+ * "fp8_kernel.py" docs, section 1.
+ *
+ *   x            device pointer, [M, N] of dtype_in, row stride ld elements.
+ *   M, N         rows and columns (0 is allowed: nothing is done).
+ *   ld           row stride of x in elements, ld >= N.
+ *   block_m/n    block shape; the pages' default weight_block_size is
+ *                [128, 128].  1 <= block_m, block_n and block_m*block_n <= 65536.
+ *   y_u8         device pointer, M*N bytes, written.
+ *   descale_f32  device pointer, ceil(M/block_m)*ceil(N/block_n) floats,
+ *                written.
+ *   stream       CUDA stream (0 = legacy default stream).
+ */
+FP8BQ_API fp8bq_status fp8bq_quantize(const void *x, fp8bq_dtype dtype_in, int64_t M, int64_t N,
+                            int64_t ld, int block_m, int block_n, uint8_t *y_u8,
+                            float *descale_f32, cudaStream_t stream);
+
+/*
+ * One tensor of a grouped call.  batch > 1 describes a stack of `batch`
+ * matrices (e.g. the experts of a fused-MoE weight [E, M, N]); each gets its
+ * own descale grid.  Matrix b starts at
+ *   x + b * x_batch_stride   (elements of dtype_in)
+ *   y + b * y_batch_stride   (bytes)
+ *   descale + b * s_batch_stride (floats).
+ * For batch == 1 the three strides are ignored.  For batch > 1 the output
+ * strides must keep the matrices apart: y_batch_stride >= M*N and
+ * s_batch_stride >= ceil(M/block_m)*ceil(N/block_n).
+ */
+typedef struct fp8bq_desc {
+    const void *x;            /* device, input */
+    uint8_t *y_u8;            /* device, e4m3fn output */
+    float *descale_f32;       /* device, fp32 descales */
+    int64_t M, N, ld;         /* rows, columns, input row stride (elements) */
+    int64_t batch;            /* number of matrices, >= 0 (1 for a plain matrix) */
+    int64_t x_batch_stride;   /* elements */
+    int64_t y_batch_stride;   /* bytes */
+    int64_t s_batch_stride;   /* floats */
+    int32_t dtype_in;         /* fp8bq_dtype */
+    int32_t block_m, block_n; /* block shape */
+    int32_t reserved;         /* set to 0 */
+} fp8bq_desc;
+
+/*
+ * Quantize a list of tensors in as few launches as possible: the
+ * quant_weights stream of the "vllm_fp8_utils.py" docs, section 3 (every
+ * linear and fused-MoE weight of a layer or a model, each emitting the fp8
+ * weight and its "_scale_inv" descale), done as one grouped launch per kernel
+ * variant instead of one launch per tensor.
+ *
+ *   desc_table   HOST memory, n_tensors entries; read during the call only.
+ *   n_tensors    >= 0.
+ *
+ * Either every tensor is checked and the whole list is enqueued, or an error
+ * is returned and nothing is launched.
+ */
+FP8BQ_API fp8bq_status fp8bq_quantize_batched(const fp8bq_desc *desc_table, int n_tensors,
+                                    cudaStream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
+
+/*
+ * Synchronize `stream`, then read and clear the library's device error word
+ * on the current device.  Returns FP8BQ_ERR_DEVICE_TIMEOUT if a kernel of this
+ * library gave up a bounded wait since the last check (its outputs are then
+ * incomplete), FP8BQ_ERR_DEVICE if the synchronization failed, else FP8BQ_OK.
+ */
+FP8BQ_API fp8bq_status fp8bq_sync_status(cudaStream_t stream);
+
+/* Library version, FP8BQ_VERSION of the build. */
+FP8BQ_API int fp8bq_version(void);
+
+/*
+ * Kernel variant selection.  AUTO picks per tensor; the others force one
+ * variant for every tensor it can serve (tensors it cannot serve still take
+ * the generic kernel).  Process-wide; meant for tests and benchmarks.
+ *   VECTOR   16-byte vectorised global loads into registers, persistent
+ *            grouped tile walk.
+ *   TMA      2-D tensor-map (TMA) tile loads into a shared-memory ring,
+ *            one producer warp, consumer warps, bounded mbarrier waits.
+ *   GENERIC  element-wise loads; any alignment, stride and block shape.
+ */
+typedef enum fp8bq_path {
+    FP8BQ_PATH_AUTO = 0,
+    FP8BQ_PATH_VECTOR = 1,
+    FP8BQ_PATH_TMA = 2,
+    FP8BQ_PATH_GENERIC = 3
+} fp8bq_path;
+
+FP8BQ_API fp8bq_status fp8bq_set_path(fp8bq_path path);
+FP8BQ_API fp8bq_path fp8bq_get_path(void);
+
+/*
+ * Which variant a tensor would take under the current selection (host only,
+ * launches nothing).  Returns FP8BQ_PATH_VECTOR, _TMA or _GENERIC, or -1 if
+ * the descriptor is invalid.
+ */
+FP8BQ_API int fp8bq_path_for(const fp8bq_desc *desc);
+
+/*
+ * Fault-injection and wait-limit knobs for tests (host side; process-wide).
+ * fp8bq_debug_set_wait_limit_ns bounds every device-side wait of the TMA
+ * kernel (default 2e9 ns; 0 restores the default).
+ * fp8bq_debug_set_inject(FP8BQ_INJECT_DROP_FIRST_LOAD) makes the first CTA of
+ * the next TMA launches arm its first tile's barrier without issuing the
+ * copy, so the consumers' wait can only run out; the kernel then reports
+ * FP8BQ_ERR_DEVICE_TIMEOUT through fp8bq_sync_status.  0 turns it off.
+ */
+#define FP8BQ_INJECT_DROP_FIRST_LOAD 1u
+FP8BQ_API fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns);
+FP8BQ_API fp8bq_status fp8bq_debug_set_inject(uint32_t flags);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BQ_H */

@@ -1,0 +1,176 @@
+"""Host-side tests of the C ABI: the library loads, exports every entry point
+the header declares, and rejects bad arguments before touching a device.
+
+These run without a GPU: argument checks happen before any CUDA call, and a
+valid call with no usable device returns FP8BQ_ERR_DEVICE.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import blockwise_fp8_weight_b200 as fq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8bq.h")
+NO_GPU = not torch.cuda.is_available()
+
+# fake, well-aligned device addresses: never dereferenced by the host checks
+X, Y, S = 0x7000_0000_0000, 0x7100_0000_0000, 0x7200_0000_0000
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"FP8BQ_API\s+[\w\s\*]+?\b(fp8bq_\w+)\s*\(", text)
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for must in ("fp8bq_quantize", "fp8bq_quantize_batched", "fp8bq_status_string",
+                 "fp8bq_sync_status"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = fq.lib()
+    for name in declared_functions():
+        assert hasattr(L, name), name
+        assert callable(getattr(L, name))
+
+
+def test_version_and_struct_layout():
+    assert fq.fp8bq_version() == 10000
+    assert ctypes.sizeof(fq.fp8bq_desc) == 96
+    assert fq.fp8bq_desc.dtype_in.offset == 80
+    assert fq.fp8bq_desc.block_n.offset == 88
+
+
+def test_status_strings():
+    for code in range(10):
+        s = fq.fp8bq_status_string(code)
+        assert s.startswith("FP8BQ_")
+    assert "unknown" in fq.fp8bq_status_string(1234)
+
+
+def q(**kw):
+    a = dict(x=X, dtype_in=fq.FP8BQ_BF16, M=256, N=384, ld=384, block_m=128, block_n=128,
+             y_u8=Y, descale_f32=S, stream=0)
+    a.update(kw)
+    return fq.fp8bq_quantize(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype_in=2), fq.FP8BQ_ERR_DTYPE),
+    (dict(dtype_in=-1), fq.FP8BQ_ERR_DTYPE),
+    (dict(block_m=0), fq.FP8BQ_ERR_BLOCK),
+    (dict(block_n=-3), fq.FP8BQ_ERR_BLOCK),
+    (dict(block_m=256, block_n=257), fq.FP8BQ_ERR_BLOCK),
+    (dict(M=-1), fq.FP8BQ_ERR_SHAPE),
+    (dict(N=-1, ld=0), fq.FP8BQ_ERR_SHAPE),
+    (dict(ld=383), fq.FP8BQ_ERR_SHAPE),
+    (dict(M=1 << 31, N=1, ld=1), fq.FP8BQ_ERR_SHAPE),
+    (dict(x=0), fq.FP8BQ_ERR_NULL),
+    (dict(y_u8=0), fq.FP8BQ_ERR_NULL),
+    (dict(descale_f32=0), fq.FP8BQ_ERR_NULL),
+    (dict(x=X + 1), fq.FP8BQ_ERR_ALIGN),
+    (dict(dtype_in=fq.FP8BQ_F32, x=X + 2), fq.FP8BQ_ERR_ALIGN),
+    (dict(descale_f32=S + 2), fq.FP8BQ_ERR_ALIGN),
+    (dict(y_u8=X + 1000), fq.FP8BQ_ERR_OVERLAP),          # y inside x
+    (dict(descale_f32=Y + 256 * 384 - 4), fq.FP8BQ_ERR_OVERLAP),  # s overlaps y's tail
+    (dict(x=Y - 2 * 384 + 2), fq.FP8BQ_ERR_OVERLAP),      # x runs into y
+])
+def test_argument_errors(kw, status):
+    assert q(**kw) == status
+
+
+def test_empty_tensors_are_a_no_op():
+    assert q(M=0, x=0, y_u8=0, descale_f32=0) == fq.FP8BQ_OK
+    assert q(N=0, ld=0) == fq.FP8BQ_OK
+    assert fq.fp8bq_quantize_batched([]) == fq.FP8BQ_OK
+
+
+@pytest.mark.skipif(not NO_GPU, reason="checks the no-device path")
+def test_valid_call_without_device_reports_device_error():
+    assert q() == fq.FP8BQ_ERR_DEVICE
+    assert q(x=X + 2) == fq.FP8BQ_ERR_DEVICE   # misaligned-for-vectors is still valid input
+
+
+def desc(**kw):
+    d = fq.fp8bq_desc()
+    a = dict(x=X, y_u8=Y, descale_f32=S, M=1536, N=2048, ld=2048, batch=128,
+             x_batch_stride=1536 * 2048, y_batch_stride=1536 * 2048, s_batch_stride=12 * 16,
+             dtype_in=fq.FP8BQ_BF16, block_m=128, block_n=128, reserved=0)
+    a.update(kw)
+    for k, v in a.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_batched_argument_errors():
+    assert fq.fp8bq_quantize_batched([desc()], n_tensors=-1) == fq.FP8BQ_ERR_ARG
+    assert fq.fp8bq_quantize_batched([desc(batch=-1)]) == fq.FP8BQ_ERR_SHAPE
+    assert fq.fp8bq_quantize_batched([desc(x_batch_stride=-5)]) == fq.FP8BQ_ERR_SHAPE
+    # experts' outputs would overlap each other
+    assert fq.fp8bq_quantize_batched([desc(y_batch_stride=1536 * 2048 - 1)]) == fq.FP8BQ_ERR_OVERLAP
+    assert fq.fp8bq_quantize_batched([desc(s_batch_stride=191)]) == fq.FP8BQ_ERR_OVERLAP
+    # two tensors writing the same output
+    a = desc()
+    b = desc(x=X + (1 << 36))
+    assert fq.fp8bq_quantize_batched([a, b]) == fq.FP8BQ_ERR_OVERLAP
+    # second tensor reads the first one's descale
+    b = desc(x=S, batch=1, M=4, N=8, ld=8, y_u8=Y + (1 << 36), descale_f32=S + (1 << 36))
+    assert fq.fp8bq_quantize_batched([a, b]) == fq.FP8BQ_ERR_OVERLAP
+    # one bad descriptor anywhere rejects the whole list
+    c = desc(x=X + (1 << 38), y_u8=Y + (1 << 38), descale_f32=S + (1 << 38), block_m=0)
+    assert fq.fp8bq_quantize_batched([a, c]) == fq.FP8BQ_ERR_BLOCK
+
+
+@pytest.mark.skipif(not NO_GPU, reason="the fake pointers must never reach a launch")
+def test_inputs_may_overlap_each_other():
+    a = desc(batch=1)
+    b = desc(batch=1, y_u8=Y + (1 << 36), descale_f32=S + (1 << 36))   # same input
+    # passes every argument check; only the missing device stops it
+    assert fq.fp8bq_quantize_batched([a, b]) == fq.FP8BQ_ERR_DEVICE
+
+
+@pytest.fixture
+def path_guard():
+    yield
+    fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
+
+
+def test_variant_choice(path_guard):
+    P = fq.fp8bq_path_for
+    assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_AUTO
+    assert P(desc()) == fq.FP8BQ_PATH_VECTOR                       # 128x128, aligned
+    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC   # rows only 8-B aligned
+    assert P(desc(batch=1, N=4096, ld=4100)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(x=X + 2)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(y_u8=Y + 4)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(batch=1, block_m=5, block_n=7)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(batch=1, block_m=256, block_n=256)) == fq.FP8BQ_PATH_GENERIC  # 65536 elements
+    assert P(desc(block_m=0)) == -1
+    assert fq.fp8bq_set_path(fq.FP8BQ_PATH_TMA) == fq.FP8BQ_OK
+    assert P(desc()) == fq.FP8BQ_PATH_TMA
+    assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
+    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC
+    assert fq.fp8bq_set_path(fq.FP8BQ_PATH_GENERIC) == fq.FP8BQ_OK
+    assert P(desc()) == fq.FP8BQ_PATH_GENERIC
+    assert fq.fp8bq_set_path(7) == fq.FP8BQ_ERR_ARG
+    assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_GENERIC
+
+
+def test_debug_knobs():
+    assert fq.fp8bq_debug_set_inject(2) == fq.FP8BQ_ERR_ARG
+    assert fq.fp8bq_debug_set_inject(0) == fq.FP8BQ_OK
+    assert fq.fp8bq_debug_set_wait_limit_ns(0) == fq.FP8BQ_OK
+
+
+@pytest.mark.skipif(not NO_GPU, reason="checks the no-device path")
+def test_sync_status_without_device():
+    assert fq.fp8bq_sync_status(0) == fq.FP8BQ_ERR_DEVICE

@@ -1,0 +1,225 @@
+"""GPU parity: every e4m3 byte and every descale bit of the CUDA library equals
+the CPU oracle, on the same seeded inputs, through the C ABI.
+
+Covers the small workload (directed blocks), the edge workload (ragged fp32
+and bf16 shapes, [1,128] and [64,64] blocks, row-padded inputs), a full
+Qwen3-8B-shaped layer, a full MoE layer with 128-expert stacks, misaligned
+pointers, degenerate shapes, each kernel variant, canary bands around every
+output, the Python conveniences, and the TMA kernel's bounded-wait error path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import blockwise_fp8_weight_b200 as fq
+import oracle
+from synth import TensorSpec, DIST_STUDENT_T3
+from synth import workloads as W
+from tests.gpu_util import assert_same, oracle_expected, run, to_device
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"auto": fq.FP8BQ_PATH_AUTO, "vector": fq.FP8BQ_PATH_VECTOR,
+         "tma": fq.FP8BQ_PATH_TMA, "generic": fq.FP8BQ_PATH_GENERIC}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+class Case:
+    """Host inputs, device inputs and oracle outputs of a list of specs."""
+
+    def __init__(self, specs):
+        self.specs = specs
+        self.host = [W.materialize(sp) for sp in specs]
+        dev = [to_device(x) for x in self.host]
+        self.owners = [o for o, _ in dev]
+        self.ptrs = [p for _, p in dev]
+        self.want = [oracle_expected(sp, x) for sp, x in zip(specs, self.host)]
+
+    def check(self, path, **kw):
+        outs = run(self.specs, self.ptrs, path, **kw)
+        for sp, o, w in zip(self.specs, outs, self.want):
+            assert_same(sp, o.result(), w)
+
+
+@pytest.fixture(scope="module")
+def small_case():
+    return Case(W.small())
+
+
+@pytest.fixture(scope="module")
+def edge_case():
+    return Case(W.edge())
+
+
+@pytest.fixture(scope="module")
+def qwen_layer_case():
+    return Case(W.qwen3_8b_layer(0, seed=1))
+
+
+@pytest.fixture(scope="module")
+def moe_layer_case():
+    return Case(W.moe_layer(0))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_small_workload(small_case, path):
+    small_case.check(PATHS[path])
+    y, s = small_case.want[0]
+    assert s[0, 1, 0] == 1.0 and s[0, 0, 1] == np.float32(np.float32(1e-10) / np.float32(448))
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_edge_workload_one_call(edge_case, path):
+    """All edge tensors (both dtypes, mixed block shapes) in one batched call."""
+    edge_case.check(PATHS[path])
+
+
+def test_edge_workload_one_call_per_tensor(edge_case):
+    for sp, p, w in zip(edge_case.specs, edge_case.ptrs, edge_case.want):
+        (o,) = run([sp], [p])
+        assert_same(sp, o.result(), w)
+
+
+@pytest.mark.parametrize("path", ["auto", "tma", "generic"])
+def test_qwen3_8b_layer(qwen_layer_case, path):
+    qwen_layer_case.check(PATHS[path])
+
+
+@pytest.mark.parametrize("path", ["auto", "tma"])
+def test_moe_layer(moe_layer_case, path):
+    moe_layer_case.check(PATHS[path])
+
+
+@pytest.mark.parametrize("dtype,xoff,yoff", [("bf16", 2, 0), ("bf16", 8, 0), ("bf16", 0, 1),
+                                             ("bf16", 0, 4), ("f32", 4, 0), ("f32", 8, 2)])
+def test_misaligned_pointers(dtype, xoff, yoff):
+    sp = TensorSpec(f"mis.{dtype}", 300, 520, dtype=dtype, seed=61, tensor_id=xoff * 10 + yoff,
+                    dist=DIST_STUDENT_T3)
+    x = W.materialize(sp)
+    owner, ptr = to_device(x, offset_bytes=xoff)
+    want = oracle_expected(sp, x)
+    for path in PATHS.values():
+        (o,) = run([sp], [ptr], path, y_offsets=[yoff])
+        assert_same(sp, o.result(), want)
+    del owner
+
+
+@pytest.mark.parametrize("shape,block", [
+    ((1, 1), (128, 128)), ((5, 5), (128, 128)), ((1, 4096), (1, 128)), ((4096, 1), (128, 128)),
+    ((7, 9), (1, 1)), ((256, 256), (256, 256)), ((300, 17), (64, 16)), ((130, 136), (2, 8)),
+    ((64, 4096), (64, 4096)), ((33, 48), (32, 16)),
+])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_degenerate_shapes_and_blocks(shape, block, dtype):
+    M, N = shape
+    if block[0] * block[1] > 65536:
+        pytest.skip("block too large by contract")
+    sp = TensorSpec(f"deg.{M}x{N}.b{block}", M, N, block=block, dtype=dtype, seed=71,
+                    tensor_id=M * 7919 + N, dist=DIST_STUDENT_T3)
+    x = W.materialize(sp)
+    owner, ptr = to_device(x)
+    want = oracle_expected(sp, x)
+    for path in PATHS.values():
+        (o,) = run([sp], [ptr], path)
+        assert_same(sp, o.result(), want)
+    del owner
+
+
+def test_all_zero_and_one_element_blocks():
+    sp = TensorSpec("zeros", 200, 264, seed=0)
+    x = np.zeros(sp.numel_storage, dtype=np.uint16)
+    x[::2] = 0x8000                                   # half the zeros are negative
+    owner, ptr = to_device(x)
+    want = oracle_expected(sp, x)
+    for path in PATHS.values():
+        (o,) = run([sp], [ptr], path)
+        y, s = o.result()
+        assert_same(sp, (y, s), want)
+        assert set(np.unique(y)) == {0x00, 0x80}
+    del owner
+
+
+def test_empty_tensor_launches_nothing():
+    d = fq.fp8bq_desc()
+    d.M, d.N, d.ld, d.batch, d.block_m, d.block_n = 0, 128, 128, 1, 128, 128
+    assert fq.fp8bq_quantize_batched([d]) == fq.FP8BQ_OK
+    assert fq.fp8bq_sync_status() == fq.FP8BQ_OK
+
+
+def test_non_default_stream_and_python_api():
+    sp = W.qwen3_8b_layer(0, seed=5)[1]               # k_proj 1024x4096
+    x = W.materialize(sp)
+    want = oracle_expected(sp, x)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(sp.M, sp.N).cuda()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        y, d = fq.scaled_fp8_blockwise(xt, [128, 128])
+    s.synchronize()
+    assert y.dtype == torch.float8_e4m3fn and y.shape == (sp.M, sp.N)
+    assert d.dtype == torch.float32 and d.shape == (8, 32)
+    assert_same(sp, (y.view(torch.uint8).cpu().numpy()[None], d.cpu().numpy()[None]), want)
+    # quant_weights: the (name, fp8), (name_scale_inv, descale) stream, one call
+    out = fq.quant_weights([("a.weight", xt), ("b.weight", xt[:512])])
+    assert [n for n, _ in out] == ["a.weight", "a.weight_scale_inv", "b.weight",
+                                   "b.weight_scale_inv"]
+    torch.cuda.synchronize()
+    assert torch.equal(out[0][1].view(torch.uint8), y.view(torch.uint8))
+    assert torch.equal(out[2][1].view(torch.uint8), y[:512].view(torch.uint8))
+    assert torch.equal(out[3][1], d[:4])
+
+
+def test_expert_stack_python_api():
+    sp = W.moe_layer(3)[5]                             # w2 [128, 2048, 768]
+    sp = TensorSpec(sp.name, sp.M, sp.N, batch=8, seed=sp.seed, tensor_id=sp.tensor_id,
+                    batch_lognormal_sigma=0.7)
+    x = W.materialize(sp)
+    want = oracle_expected(sp, x)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).reshape(8, sp.M, sp.N).cuda()
+    y, d = fq.scaled_fp8_blockwise(xt)
+    torch.cuda.synchronize()
+    assert y.shape == (8, 2048, 768) and d.shape == (8, 16, 6)
+    assert_same(sp, (y.view(torch.uint8).cpu().numpy(), d.cpu().numpy()), want)
+
+
+def test_variant_bytes_agree_on_large_input(qwen_layer_case):
+    """The vector and TMA variants write identical bytes on a full layer."""
+    a = run(qwen_layer_case.specs, qwen_layer_case.ptrs, fq.FP8BQ_PATH_VECTOR)
+    b = run(qwen_layer_case.specs, qwen_layer_case.ptrs, fq.FP8BQ_PATH_TMA)
+    for oa, ob in zip(a, b):
+        assert torch.equal(oa.y.view, ob.y.view) and torch.equal(oa.s.view, ob.s.view)
+
+
+def test_tma_bounded_wait_reports_timeout_and_recovers():
+    """The first CTA arms its first barrier without issuing the copy, so its
+    consumers' wait can only run out: the kernel must return, report
+    FP8BQ_ERR_DEVICE_TIMEOUT, and leave the context usable."""
+    sp = W.qwen3_8b_layer(0, seed=9)[0]                # q_proj 4096x4096
+    x = W.materialize(sp)
+    owner, ptr = to_device(x)
+    want = oracle_expected(sp, x)
+    assert fq.fp8bq_debug_set_wait_limit_ns(5_000_000) == fq.FP8BQ_OK   # 5 ms
+    assert fq.fp8bq_debug_set_inject(fq.FP8BQ_INJECT_DROP_FIRST_LOAD) == fq.FP8BQ_OK
+    try:
+        from tests.gpu_util import Outputs
+        o = Outputs(sp)
+        fq.fp8bq_set_path(fq.FP8BQ_PATH_TMA)
+        assert fq.fp8bq_quantize_batched([o.desc(ptr)]) == fq.FP8BQ_OK
+        assert fq.fp8bq_sync_status() == fq.FP8BQ_ERR_DEVICE_TIMEOUT
+        assert fq.fp8bq_sync_status() == fq.FP8BQ_OK          # the word was cleared
+        assert o.y.canaries_intact() and o.s.canaries_intact()
+    finally:
+        fq.fp8bq_debug_set_inject(0)
+        fq.fp8bq_debug_set_wait_limit_ns(0)
+        fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
+    (o2,) = run([sp], [ptr], fq.FP8BQ_PATH_TMA)
+    assert_same(sp, o2.result(), want)
+    del owner
