@@ -42,16 +42,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not verbose_ptxas and up_to_date():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str | None = None,
+          defines: tuple[str, ...] = ()) -> str:
+    """Compile the library (to ``out``, default the in-tree path); ``defines``
+    are extra -D tuning constants."""
+    lib = out or LIB
+    if out is None and not force and not verbose_ptxas and not defines and up_to_date():
         return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *SOURCES]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *ARCH, *FLAGS, *(f"-D{d}" for d in defines), "-I", os.path.join(ROOT, "include"),
+           "-o", tmp, *SOURCES]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -156,14 +156,28 @@ bool tma_fits(const fp8bq_desc &D) {
     return vector_aligned(D);
 }
 
+// AUTO: the TMA ring for blocks of at least 8 KB (one ring slot per block
+// keeps enough bytes in flight), the register-tile vector kernel for smaller
+// aligned blocks, the generic kernel for everything else.
+constexpr int64_t kTmaMinBlockBytes = 8192;
+
 Variant choose(const fp8bq_desc &D, int path) {
     if (path == FP8BQ_PATH_GENERIC) return Variant::Generic;
     if (path == FP8BQ_PATH_TMA && tma_fits(D)) return Variant::Tma;
+    if (path == FP8BQ_PATH_AUTO && tma_fits(D) &&
+        (int64_t)D.block_m * D.block_n * esize_of(D.dtype_in) >= kTmaMinBlockBytes)
+        return Variant::Tma;
     if (!vector_aligned(D)) return Variant::Generic;
     return vector_variant(D);
 }
 
 // ------------------------------------------------------------------ tensor maps
+
+// L2 promotion of the TMA tile loads (CUtensorMapL2promotion: 0 none, 1 64 B,
+// 2 128 B, 3 256 B); a tile row is 256 bytes of bf16.
+#ifndef FP8BQ_TMA_L2_PROMOTION
+#define FP8BQ_TMA_L2_PROMOTION 3
+#endif
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
@@ -231,7 +245,7 @@ bool encode_map(const fp8bq_desc &D, CUtensorMap *out) {
                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                     3, const_cast<void *>(D.x), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    (CUtensorMapL2promotion)FP8BQ_TMA_L2_PROMOTION, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return false;
     std::lock_guard<std::mutex> g(mu);
     if (cache.size() > 8192) cache.clear();

@@ -29,20 +29,77 @@ __device__ __forceinline__ void stg_stream_u32(void *p, uint32_t v) {
     asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// ---------------------------------------------------------------- arithmetic
+// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned address) into L2.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
-// Two fp32 values -> two e4m3fn codes, round to nearest even, saturating to
-// +-448; `lo` lands in the low byte (the lower address).
+// ---------------------------------------------------------------- arithmetic
+//
+// The clamp of the method, clamp(x * r, -448, 448), is not issued as separate
+// min/max instructions: cvt.rn.satfinite maps every finite value beyond the
+// e4m3fn range to +-448 and rounds every value inside it to nearest even, so
+// e4m3(clamp(v)) == cvt.rn.satfinite(v) for every finite v (and v = x * r is
+// always finite: |x| <= absmax and r ~ 448 / absmax).
+
+// Two fp32 values -> two e4m3fn codes (round to nearest even, saturating);
+// `lo` lands in the low byte (the lower address).
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return (uint32_t)r;
 }
 
-// One quantized element: clamp(x * r, -448, 448), single-rounded multiply.
-__device__ __forceinline__ float scale_clamp(float x, float r) {
-    float v = __fmul_rn(x, r);
-    return fminf(fmaxf(v, -448.0f), 448.0f);
+// A register pair {r, r} for the packed multiplies of one block.
+__device__ __forceinline__ uint64_t splat2(float r) {
+    uint64_t d;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(d) : "f"(r));
+    return d;
+}
+
+// Codes of the two fp32 values whose bit patterns are a0, a1: one packed
+// single-rounded multiply (each lane IEEE round-to-nearest, no FMA, no
+// flush-to-zero) and one conversion.  a0 lands in the low byte.
+__device__ __forceinline__ uint16_t quant_pair_bits(uint32_t a0, uint32_t a1, uint64_t rr) {
+    uint64_t a, d;
+    uint16_t h;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "r"(a0), "r"(a1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(rr));
+    asm("{\n\t.reg .f32 v0, v1;\n\t"
+        "mov.b64 {v0, v1}, %1;\n\t"
+        "cvt.rn.satfinite.e4m3x2.f32 %0, v1, v0;\n\t}"
+        : "=h"(h)
+        : "l"(d));
+    return h;
+}
+
+// Four bf16 (two 32-bit words, element order w0.lo, w0.hi, w1.lo, w1.hi) ->
+// four codes in one 32-bit word, element 0 in the low byte.
+__device__ __forceinline__ uint32_t quant_bf16x4(uint32_t w0, uint32_t w1, uint64_t rr) {
+    const uint16_t c0 = quant_pair_bits(w0 << 16, w0 & 0xffff0000u, rr);
+    const uint16_t c1 = quant_pair_bits(w1 << 16, w1 & 0xffff0000u, rr);
+    uint32_t o;
+    asm("mov.b32 %0, {%1, %2};" : "=r"(o) : "h"(c0), "h"(c1));
+    return o;
+}
+
+// Four fp32 (bit patterns) -> four codes in one 32-bit word.
+__device__ __forceinline__ uint32_t quant_f32x4(uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                                uint64_t rr) {
+    const uint16_t c0 = quant_pair_bits(a, b, rr);
+    const uint16_t c1 = quant_pair_bits(c, d, rr);
+    uint32_t o;
+    asm("mov.b32 %0, {%1, %2};" : "=r"(o) : "h"(c0), "h"(c1));
+    return o;
+}
+
+// Running max of the magnitudes of two packed bf16 (unsigned halfword max of
+// the sign-cleared bit patterns: for non-negative IEEE values the integer
+// order of the bits is the numeric order).
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(w & 0x7fff7fffu));
+    return d;
 }
 
 // bf16 halves of a 32-bit word, widened to fp32 (exact).

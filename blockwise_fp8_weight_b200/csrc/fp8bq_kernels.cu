@@ -31,6 +31,23 @@ __device__ uint32_t g_error_word;
 
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
+// Tuning constants (compile-time; the defaults are the measured best on B200).
+#ifndef FP8BQ_VEC_CTAS_PER_SM
+#define FP8BQ_VEC_CTAS_PER_SM 2   // resident 256-thread vector CTAs per SM
+#endif
+#ifndef FP8BQ_VEC_L2_PREFETCH
+#define FP8BQ_VEC_L2_PREFETCH 0   // vector kernel: bulk-prefetch the tile after next into L2
+#endif
+#ifndef FP8BQ_TMA_STAGES_BF16
+#define FP8BQ_TMA_STAGES_BF16 6   // 32 KB ring slots per TMA CTA (bf16 tiles)
+#endif
+#ifndef FP8BQ_TMA_STAGES_F32
+#define FP8BQ_TMA_STAGES_F32 3    // 64 KB ring slots per TMA CTA (fp32 tiles)
+#endif
+#ifndef FP8BQ_TMA_CTAS_PER_SM
+#define FP8BQ_TMA_CTAS_PER_SM 1   // resident TMA CTAs per SM
+#endif
+
 // Tile geometry shared by all kernels.
 struct Tile {
     const char *src;  // first element of the block
@@ -71,10 +88,10 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
 template <int ESIZE>
 __device__ __forceinline__ uint32_t vec_absmax(const uint4 &v, uint32_t m) {
     if constexpr (ESIZE == 2) {
-        m = __vmaxu2(m, v.x & 0x7fff7fffu);
-        m = __vmaxu2(m, v.y & 0x7fff7fffu);
-        m = __vmaxu2(m, v.z & 0x7fff7fffu);
-        m = __vmaxu2(m, v.w & 0x7fff7fffu);
+        m = dev::absmax_bf16x2(m, v.x);
+        m = dev::absmax_bf16x2(m, v.y);
+        m = dev::absmax_bf16x2(m, v.z);
+        m = dev::absmax_bf16x2(m, v.w);
     } else {
         m = max(m, v.x & 0x7fffffffu);
         m = max(m, v.y & 0x7fffffffu);
@@ -93,29 +110,17 @@ __device__ __forceinline__ uint32_t absmax_to_f32_bits(uint32_t m) {
         return m;
 }
 
-// Quantize one 16-byte vector and store its codes (8 bytes for bf16, 4 for fp32).
+// Quantize one 16-byte vector with rr = {r, r} and store its codes (8 bytes
+// for bf16, 4 for fp32).
 template <int ESIZE>
-__device__ __forceinline__ void vec_quant_store(const uint4 &v, float r, uint8_t *dst) {
+__device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uint8_t *dst) {
     if constexpr (ESIZE == 2) {
         uint2 o;
-        o.x = dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.x), r),
-                              dev::scale_clamp(dev::bf16_hi(v.x), r)) |
-              (dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.y), r),
-                               dev::scale_clamp(dev::bf16_hi(v.y), r))
-               << 16);
-        o.y = dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.z), r),
-                              dev::scale_clamp(dev::bf16_hi(v.z), r)) |
-              (dev::cvt_e4m3x2(dev::scale_clamp(dev::bf16_lo(v.w), r),
-                               dev::scale_clamp(dev::bf16_hi(v.w), r))
-               << 16);
+        o.x = dev::quant_bf16x4(v.x, v.y, rr);
+        o.y = dev::quant_bf16x4(v.z, v.w, rr);
         dev::stg_stream_v2(dst, o);
     } else {
-        uint32_t o = dev::cvt_e4m3x2(dev::scale_clamp(__uint_as_float(v.x), r),
-                                     dev::scale_clamp(__uint_as_float(v.y), r)) |
-                     (dev::cvt_e4m3x2(dev::scale_clamp(__uint_as_float(v.z), r),
-                                      dev::scale_clamp(__uint_as_float(v.w), r))
-                      << 16);
-        dev::stg_stream_u32(dst, o);
+        dev::stg_stream_u32(dst, dev::quant_f32x4(v.x, v.y, v.z, v.w, rr));
     }
 }
 
@@ -129,7 +134,7 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, float r, uint8_t
 // segments.  bm and bn are the same for every tensor of a launch.
 
 template <int ESIZE, int TEAM, int V, int CTA, int MAXD>
-__global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
+__global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
@@ -149,6 +154,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
     const int colv = cv * VEC;
     const uint32_t shfl_mask =
         TEAM >= 32 ? 0xffffffffu : (((1u << TEAM) - 1u) << ((threadIdx.x & 31) & ~(TEAM - 1)));
+    int d = 0;  // current descriptor; advances monotonically with the tile id
 
     auto load = [&](uint4 (&R)[V], const Tile &T) {
 #pragma unroll
@@ -159,6 +165,15 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
             else
                 R[i] = make_uint4(0u, 0u, 0u, 0u);
         }
+    };
+
+    // Bulk-prefetch the rows of tile tn into L2 (a hint; no data dependence).
+    auto prefetch = [&](uint32_t tn) {
+        if (!FP8BQ_VEC_L2_PREFETCH || tn >= p.total_tiles) return;
+        int dd = d;
+        const Tile T = make_tile<ESIZE>(p, tn, dd);
+        for (int r = lane; r < T.rows; r += TEAM)
+            dev::prefetch_l2(T.src + (int64_t)r * T.ld * ESIZE, (uint32_t)(T.cols * ESIZE));
     };
 
     auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
@@ -179,16 +194,16 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
         }
         float s, r;
         dev::block_scale(m, kEps, s, r);
+        const uint64_t r2 = dev::splat2(r);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int rr = row0 + i * rstep;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], r, T.dst + (int64_t)rr * T.ldy + colv);
+                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
         }
         if (lane == 0) *T.sdst = s;
     };
 
-    int d = 0;
     uint4 A[V], B[V];
     Tile ta = make_tile<ESIZE>(p, t, d);
     load(A, ta);
@@ -200,6 +215,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
         if (h1) {
             tb = make_tile<ESIZE>(p, t1, d);
             load(B, tb);
+            prefetch(t1 + stride);
         }
         process(A, ta, it++);
         if (!h1) break;
@@ -208,6 +224,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? 2 : 1))
         if (h2) {
             ta = make_tile<ESIZE>(p, t2, d);
             load(A, ta);
+            prefetch(t2 + stride);
         }
         process(B, tb, it++);
         if (!h2) break;
@@ -256,7 +273,7 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
             const char *row = T.src + (int64_t)r * T.ld * ESIZE;
             uint8_t *out = T.dst + (int64_t)r * T.ldy;
             for (int c = lane; c < T.cols; c += 32) {
-                const float v = dev::scale_clamp(elem_f32<ESIZE>(row + c * ESIZE), rc);
+                const float v = __fmul_rn(elem_f32<ESIZE>(row + c * ESIZE), rc);
                 out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
             }
         }
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
 // (bounded) for each copy it issued before it returns.
 
 template <int ESIZE, int STAGES>
-__global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
+__global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
     k_tma(const __grid_constant__ TmaPack<kMaxDescTma> P) {
     constexpr int VEC = 16 / ESIZE;
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
@@ -383,11 +400,12 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
         for (int w = 1; w < kTmaConsumerThreads / 32; ++w) m = max(m, red[k & 1][w]);
         float s, r;
         dev::block_scale(m, kEps, s, r);
+        const uint64_t r2 = dev::splat2(r);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int rr = row0 + i * rstep;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], r, T.dst + (int64_t)rr * T.ldy + colv);
+                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
         }
         if (ct == 0) *T.sdst = s;
     }
@@ -479,7 +497,8 @@ cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
-    return esize == 2 ? launch_tma_t<2, 6>(p, st) : launch_tma_t<4, 3>(p, st);
+    return esize == 2 ? launch_tma_t<2, FP8BQ_TMA_STAGES_BF16>(p, st)
+                      : launch_tma_t<4, FP8BQ_TMA_STAGES_F32>(p, st);
 }
 
 cudaError_t read_and_clear_error_word(uint32_t *out) {

@@ -144,10 +144,14 @@ def path_guard():
 def test_variant_choice(path_guard):
     P = fq.fp8bq_path_for
     assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_AUTO
-    assert P(desc()) == fq.FP8BQ_PATH_VECTOR                       # 128x128, aligned
-    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR
-    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_VECTOR
-    assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc()) == fq.FP8BQ_PATH_TMA                          # 128x128, aligned
+    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR   # 256-B blocks
+    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_TMA      # 8 KB blocks
+    assert P(desc(batch=1, block_m=32, block_n=64)) == fq.FP8BQ_PATH_VECTOR   # 4 KB blocks
+    assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
+    assert fq.fp8bq_set_path(fq.FP8BQ_PATH_VECTOR) == fq.FP8BQ_OK
+    assert P(desc()) == fq.FP8BQ_PATH_VECTOR
+    assert fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO) == fq.FP8BQ_OK
     assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC   # rows only 8-B aligned
     assert P(desc(batch=1, N=4096, ld=4100)) == fq.FP8BQ_PATH_GENERIC
     assert P(desc(x=X + 2)) == fq.FP8BQ_PATH_GENERIC
