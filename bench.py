@@ -113,6 +113,9 @@ def workload(name: str):
                                 "and w2 stacks, bf16, block 128x128, one grouped launch")
     if name == "small":
         return W.small(), "256x384 bf16, 2x3 blocks of 128x128"
+    if name == "qkv":
+        return W.qkv_activations(), ("Q/K/V activations of one Qwen3-8B-shaped attention layer, "
+                                     "16384 tokens, bf16 (per-tensor scale recalibration)")
     if name in ("act_1x128", "blk_64x64"):
         sp = [t for t in W.edge() if t.name.endswith("b1x128" if name == "act_1x128" else "b64x64")]
         return sp, f"bf16 16384x4096, N(0,1) x row lognormal(0,1), blocks {sp[0].block}"
@@ -185,16 +188,16 @@ def host_inputs(specs, lay: Layout, local_rank: int, dist: Dist, tag: str):
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons with NVML while running."""
+    """Samples SM clock, power and clock-event reasons with NVML while running."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
                0x8: "hw_slowdown", 0x20: "sync_boost", 0x40: "sw_thermal_slowdown",
                0x80: "hw_thermal_slowdown", 0x100: "hw_power_brake_slowdown",
                0x200: "display_clock_setting"}
 
-    def __init__(self, torch_device, period_s=0.005):
+    def __init__(self, torch_device, period_s=0.004):
         self.period = period_s
-        self.samples, self.reasons = [], 0
+        self.samples, self.power, self.reason_samples = [], [], []
         self.max_mhz = None
         self._stop = threading.Event()
         self._thr = None
@@ -220,7 +223,8 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= self._reasons_now()
+                self.reason_samples.append(self._reasons_now())
+                self.power.append(self.nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
             except Exception:
                 pass
             time.sleep(self.period)
@@ -239,9 +243,15 @@ class ClockSampler:
     def summary(self) -> dict:
         if self.nv is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
-        med = float(np.median(self.samples)) if self.samples else None
-        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
-                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b]}
+        n = len(self.reason_samples)
+        frac = {name: round(sum(1 for r in self.reason_samples if r & bit) / n, 3)
+                for bit, name in self.REASONS.items()
+                if n and any(r & bit for r in self.reason_samples)}
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_min_mhz": min(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "samples": len(self.samples),
+                "power_w_median": float(np.median(self.power)) if self.power else None,
+                "reasons": sorted(frac), "reason_sample_fraction": frac}
 
 
 def measured_peak() -> tuple[float, str]:
@@ -443,6 +453,25 @@ def run_ours(args) -> None:
     max_elapsed = dist.max(elapsed_s)
     value = aggregate(bytes_per_step, args.steps, world, max_elapsed)
 
+    if args.op in ("dequantize", "tensor_scale"):
+        if args.op == "dequantize":
+            run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_desc)
+        else:
+            run_scale_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc)
+        fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
+        if pinned_in:
+            cudart.cudaHostUnregister(hptr)
+        del host_t, host
+        dist.barrier()
+        if local_rank == 0 and not args.keep_inputs:
+            for pth in (shm_path, shm_path + ".done"):
+                try:
+                    os.remove(pth)
+                except OSError:
+                    pass
+        dist.close()
+        return
+
     # ---- end to end: inputs from pinned host memory, outputs back to host memory
     y_host = torch.empty(lay.y_bytes, dtype=torch.uint8, pin_memory=True)
     s_host = torch.empty(lay.s_bytes, dtype=torch.uint8, pin_memory=True)
@@ -561,6 +590,127 @@ def run_ours(args) -> None:
     dist.close()
 
 
+def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_desc) -> None:
+    """Time fp8bq_dequantize_batched (bf16 output) over every quantized tensor
+    of the workload, one grouped call per step; the codes come from the
+    quantize steps already run."""
+    import torch
+    import blockwise_fp8_weight_b200 as fq
+    out_off, o = [], 0
+    for sp in specs:
+        out_off.append(o)
+        o = align(o + sp.numel * 2, 256)
+    out = torch.empty(o, dtype=torch.uint8, device=dev)
+    L = fq.lib()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+    table = (fq.fp8bq_dequant_desc * len(specs))()
+    for i, sp in enumerate(specs):
+        d = table[i]
+        d.y_u8 = y_dev.data_ptr() + lay.y_off[i]
+        d.descale_f32 = s_dev.data_ptr() + lay.s_off[i]
+        d.out = out.data_ptr() + out_off[i]
+        d.batch, d.M, d.N = sp.batch, sp.M, sp.N
+        d.ld_out, d.out_batch_stride = sp.N, sp.M * sp.N
+        d.dtype_out = fq.FP8BQ_BF16
+        d.block_m, d.block_n = sp.block
+        d.reserved = 0
+
+    def step():
+        st = L.fp8bq_dequantize_batched(table, len(specs), sh)
+        if st != 0:
+            raise RuntimeError(fq.fp8bq_status_string(st))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with ClockSampler(dev) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        while not t1.query():
+            time.sleep(0.0005)
+        torch.cuda.synchronize()
+    dist.barrier()
+    el = dist.max(t0.elapsed_time(t1) / 1e3)
+    nbytes = sum(sp.numel * 3 + sp.nblocks * 4 for sp in specs)
+    value = aggregate(nbytes, args.steps, world, el)
+    peak, kind = measured_peak()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "blockwise FP8 dequantize GB/s (e4m3 codes + descales in, bf16 out)",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl_desc + " (dequantize its codes to bf16)",
+                       "name": args.workload, "op": "dequantize", "bytes_per_step": nbytes,
+                       "launches_per_step": -(-len(specs) // 320)},
+            "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
+                         "frac": value / world / peak, "traffic": None,
+                         "peak_source": kind},
+            "gpu_launches": -(-len(specs) // 320) * args.steps, "clocks": clk.summary()}),
+              flush=True)
+
+
+def run_scale_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc) -> None:
+    """Time fp8bq_tensor_scale over every tensor of the workload (one grouped
+    call per step): a read-only pass, numel * elem_bytes + 4 bytes per tensor."""
+    import torch
+    import blockwise_fp8_weight_b200 as fq
+    table = (fq.fp8bq_scale_desc * len(specs))()
+    for i, sp in enumerate(specs):
+        table[i].x = x_dev.data_ptr() + lay.x_off[i]
+        table[i].numel = sp.numel_storage
+        table[i].dtype_in = fq.FP8BQ_BF16 if sp.dtype == "bf16" else fq.FP8BQ_F32
+        table[i].reserved = 0
+    out = torch.empty(len(specs), dtype=torch.float32, device=dev)
+    L = fq.lib()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+
+    def step():
+        st = L.fp8bq_tensor_scale(table, len(specs), ctypes.c_void_p(out.data_ptr()), sh)
+        if st != 0:
+            raise RuntimeError(fq.fp8bq_status_string(st))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    with ClockSampler(dev) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        while not t1.query():
+            time.sleep(0.0005)
+        torch.cuda.synchronize()
+    dist.barrier()
+    el = dist.max(t0.elapsed_time(t1) / 1e3)
+    nbytes = sum(sp.numel_storage * sp.elem_bytes + 4 for sp in specs)
+    value = aggregate(nbytes, args.steps, world, el)
+    peak, kind = measured_peak()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "per-tensor FP8 scale GB/s (bytes read)", "value": value, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl_desc, "name": args.workload, "op": "tensor_scale",
+                       "bytes_per_step": nbytes, "tensors": len(specs)},
+            "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
+                         "frac": value / world / peak, "traffic": None, "peak_source": kind,
+                         "note": "one memset, one grid-wide pass and one finalize launch per step"},
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}), flush=True)
+
+
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -569,9 +719,13 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_model",
                     choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small",
-                             "act_1x128", "blk_64x64"])
+                             "act_1x128", "blk_64x64", "qkv"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale"],
+                    default="quantize",
+                    help="dequantize: time the reverse map on the quantized workload; "
+                         "tensor_scale: time per-tensor scales of the workload's tensors")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time spent on the oracle baseline (0 = skip)")
     ap.add_argument("--keep-inputs", action="store_true",

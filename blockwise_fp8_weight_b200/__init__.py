@@ -68,6 +68,27 @@ class fp8bq_desc(ctypes.Structure):
     ]
 
 
+class fp8bq_dequant_desc(ctypes.Structure):
+    """Mirror of ``struct fp8bq_dequant_desc`` (80 bytes)."""
+    _fields_ = [
+        ("y_u8", ctypes.c_void_p),
+        ("descale_f32", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("batch", ctypes.c_int64), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("ld_out", ctypes.c_int64),
+        ("out_batch_stride", ctypes.c_int64),
+        ("dtype_out", ctypes.c_int32),
+        ("block_m", ctypes.c_int32), ("block_n", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class fp8bq_scale_desc(ctypes.Structure):
+    """Mirror of ``struct fp8bq_scale_desc`` (24 bytes)."""
+    _fields_ = [("x", ctypes.c_void_p), ("numel", ctypes.c_int64),
+                ("dtype_in", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 class Fp8bqError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
@@ -94,6 +115,12 @@ def lib() -> ctypes.CDLL:
             L.fp8bq_quantize.restype = i32
             L.fp8bq_quantize_batched.argtypes = [ctypes.POINTER(fp8bq_desc), i32, vp]
             L.fp8bq_quantize_batched.restype = i32
+            L.fp8bq_dequantize.argtypes = [vp, vp, i64, i64, i64, i32, i32, vp, i32, i64, i64, vp]
+            L.fp8bq_dequantize.restype = i32
+            L.fp8bq_dequantize_batched.argtypes = [ctypes.POINTER(fp8bq_dequant_desc), i32, vp]
+            L.fp8bq_dequantize_batched.restype = i32
+            L.fp8bq_tensor_scale.argtypes = [ctypes.POINTER(fp8bq_scale_desc), i32, vp, vp]
+            L.fp8bq_tensor_scale.restype = i32
             L.fp8bq_status_string.argtypes = [i32]
             L.fp8bq_status_string.restype = ctypes.c_char_p
             L.fp8bq_sync_status.argtypes = [vp]
@@ -152,6 +179,30 @@ def fp8bq_quantize_batched(desc_table: Sequence[fp8bq_desc] | ctypes.Array, n_te
         desc_table = (fp8bq_desc * len(desc_table))(*desc_table)
     n = len(desc_table) if n_tensors is None else n_tensors
     return lib().fp8bq_quantize_batched(desc_table, n, _stream(stream))
+
+
+def fp8bq_dequantize(y_u8, descale_f32, batch: int, M: int, N: int, block_m: int, block_n: int,
+                     out, dtype_out: int, ld_out: int, out_batch_stride: int, stream=None) -> int:
+    """``fp8bq_dequantize`` of the C ABI.  Returns the status code."""
+    return lib().fp8bq_dequantize(_ptr(y_u8), _ptr(descale_f32), batch, M, N, block_m, block_n,
+                                  _ptr(out), dtype_out, ld_out, out_batch_stride,
+                                  _stream(stream))
+
+
+def fp8bq_dequantize_batched(desc_table, n_tensors=None, stream=None) -> int:
+    """``fp8bq_dequantize_batched`` of the C ABI.  Returns the status code."""
+    if not isinstance(desc_table, ctypes.Array):
+        desc_table = (fp8bq_dequant_desc * len(desc_table))(*desc_table)
+    n = len(desc_table) if n_tensors is None else n_tensors
+    return lib().fp8bq_dequantize_batched(desc_table, n, _stream(stream))
+
+
+def fp8bq_tensor_scale(desc_table, scale_out, n_tensors=None, stream=None) -> int:
+    """``fp8bq_tensor_scale`` of the C ABI.  Returns the status code."""
+    if not isinstance(desc_table, ctypes.Array):
+        desc_table = (fp8bq_scale_desc * len(desc_table))(*desc_table)
+    n = len(desc_table) if n_tensors is None else n_tensors
+    return lib().fp8bq_tensor_scale(desc_table, n, _ptr(scale_out), _stream(stream))
 
 
 def fp8bq_status_string(status: int) -> str:
@@ -248,6 +299,46 @@ def scaled_fp8_blockwise(data_hp, weight_block_size=DEFAULT_BLOCK, stream=None):
     check(fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream),
           "scaled_fp8_blockwise")
     return y, s
+
+
+def dequantize_fp8_blockwise(fp8_data, descale, weight_block_size=DEFAULT_BLOCK,
+                             out_dtype=None, stream=None):
+    """Reverse map of ``scaled_fp8_blockwise``: decode(fp8_data) * descale per
+    block, as bf16 (default) or fp32, same shape as ``fp8_data``."""
+    import torch
+    out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    if not fp8_data.is_contiguous() or not descale.is_contiguous():
+        raise ValueError("fp8_data and descale must be contiguous")
+    bm, bn = (int(b) for b in weight_block_size)
+    M, N = fp8_data.shape[-2], fp8_data.shape[-1]
+    batch = fp8_data.shape[0] if fp8_data.dim() == 3 else 1
+    out = torch.empty(fp8_data.shape, dtype=out_dtype, device=fp8_data.device)
+    check(fp8bq_dequantize(fp8_data, descale, batch, M, N, bm, bn, out,
+                           FP8BQ_BF16 if out_dtype == torch.bfloat16 else FP8BQ_F32, N, M * N,
+                           stream), "dequantize_fp8_blockwise")
+    return out
+
+
+def tensor_scales(tensors, stream=None):
+    """Per-tensor FP8 scales max(max|x|, eps) / 448 of contiguous bf16/fp32
+    CUDA tensors (e.g. this step's Q, K and V), in one grouped call; returns a
+    float32 CUDA tensor of len(tensors) scales."""
+    import torch
+    tensors = list(tensors)
+    if not tensors:
+        raise ValueError("no tensors")
+    out = torch.empty(len(tensors), dtype=torch.float32, device=tensors[0].device)
+    descs = []
+    for t in tensors:
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        d = fp8bq_scale_desc()
+        d.x, d.numel, d.dtype_in, d.reserved = _ptr(t), t.numel(), _dtype_code(t), 0
+        descs.append(d)
+    check(fp8bq_tensor_scale(descs, out, stream=stream), "tensor_scales")
+    return out
 
 
 def quant_weights(weights: Iterable, weight_block_size=DEFAULT_BLOCK, stream=None):

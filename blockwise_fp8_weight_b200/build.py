@@ -16,7 +16,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, f) for f in ("fp8bq_api.cu", "fp8bq_kernels.cu")]
+SOURCES = [os.path.join(CSRC, f) for f in ("fp8bq_api.cu", "fp8bq_kernels.cu", "fp8bq_dequant.cu",
+                                                   "fp8bq_scale.cu")]
 HEADERS = [os.path.join(CSRC, f) for f in ("fp8bq_internal.h", "fp8bq_device.cuh")] + [
     os.path.join(ROOT, "include", "fp8bq.h")]
 LIB = os.path.join(PKG, "libfp8bq.so")

@@ -125,6 +125,7 @@ bool vector_fits(const fp8bq_desc &D, Variant v) {
     if (D.block_n % vec) return false;
     const int vpr = D.block_n / vec;
     if (!is_pow2(vpr) || vpr > team) return false;
+    if (v == Variant::VecT16) return (int64_t)D.block_m * vpr == team;  // one row-step per block
     return cdiv(D.block_m, team / vpr) <= slots;
 }
 
@@ -156,10 +157,10 @@ bool tma_fits(const fp8bq_desc &D) {
     return vector_aligned(D);
 }
 
-// AUTO: the TMA ring for blocks of at least 8 KB (one ring slot per block
-// keeps enough bytes in flight), the register-tile vector kernel for smaller
-// aligned blocks, the generic kernel for everything else.
-constexpr int64_t kTmaMinBlockBytes = 8192;
+// AUTO: the TMA ring for blocks of at least 32 KB (one ring slot holds one
+// block, so smaller blocks leave too few bytes in flight), the register-tile
+// vector kernel for smaller aligned blocks, the generic kernel otherwise.
+constexpr int64_t kTmaMinBlockBytes = 32768;
 
 Variant choose(const fp8bq_desc &D, int path) {
     if (path == FP8BQ_PATH_GENERIC) return Variant::Generic;
@@ -256,7 +257,11 @@ bool encode_map(const fp8bq_desc &D, CUtensorMap *out) {
 
 // ------------------------------------------------------------------ launches
 
-void fill_tile_desc(const fp8bq_desc &D, uint32_t begin, TileDesc *o) {
+uint64_t tiles_of(const fp8bq_desc &D, Variant v) {
+    return (uint64_t)D.batch * cdiv(cdiv(D.M, D.block_m), kTileBlocksM(v)) * cdiv(D.N, D.block_n);
+}
+
+void fill_tile_desc(const fp8bq_desc &D, Variant v, uint32_t begin, TileDesc *o) {
     o->x = D.x;
     o->y = D.y_u8;
     o->s = D.descale_f32;
@@ -271,7 +276,7 @@ void fill_tile_desc(const fp8bq_desc &D, uint32_t begin, TileDesc *o) {
     o->gm = (int32_t)cdiv(D.M, D.block_m);
     o->gn = (int32_t)cdiv(D.N, D.block_n);
     o->tile_begin = begin;
-    o->tiles = (uint32_t)(D.batch * o->gm * o->gn);
+    o->tiles = (uint32_t)tiles_of(D, v);
 }
 
 template <int MAXD>
@@ -294,9 +299,9 @@ cudaError_t launch_group(Variant v, int es, const fp8bq_desc *t, const std::vect
         pack_header(p);
         while (i < idx.size() && p.n < MAXD) {
             const fp8bq_desc &D = t[idx[i]];
-            const uint64_t tiles = (uint64_t)D.batch * cdiv(D.M, D.block_m) * cdiv(D.N, D.block_n);
+            const uint64_t tiles = tiles_of(D, v);
             if (p.n > 0 && (uint64_t)p.total_tiles + tiles >= (1ull << 31)) break;
-            fill_tile_desc(D, p.total_tiles, &p.d[p.n]);
+            fill_tile_desc(D, v, p.total_tiles, &p.d[p.n]);
             p.total_tiles += (uint32_t)tiles;
             ++p.n;
             ++i;
@@ -316,9 +321,9 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
         pack_header(P.p);
         while (i < idx.size() && P.p.n < kMaxDescTma) {
             const fp8bq_desc &D = t[idx[i]];
-            const uint64_t tiles = (uint64_t)D.batch * cdiv(D.M, D.block_m) * cdiv(D.N, D.block_n);
+            const uint64_t tiles = tiles_of(D, Variant::Tma);
             if (P.p.n > 0 && (uint64_t)P.p.total_tiles + tiles >= (1ull << 31)) break;
-            fill_tile_desc(D, P.p.total_tiles, &P.p.d[P.p.n]);
+            fill_tile_desc(D, Variant::Tma, P.p.total_tiles, &P.p.d[P.p.n]);
             P.maps[P.p.n] = maps[i];
             P.p.total_tiles += (uint32_t)tiles;
             ++P.p.n;
@@ -392,9 +397,206 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
     return FP8BQ_OK;
 }
 
+// ------------------------------------------------------------------ dequantization
+
+fp8bq_status check_dequant_desc(const fp8bq_dequant_desc &D, bool *empty) {
+    if (D.dtype_out != FP8BQ_BF16 && D.dtype_out != FP8BQ_F32) return FP8BQ_ERR_DTYPE;
+    if (D.block_m < 1 || D.block_n < 1 || (int64_t)D.block_m * D.block_n > 65536)
+        return FP8BQ_ERR_BLOCK;
+    if (D.batch < 0 || D.M < 0 || D.N < 0 || D.ld_out < D.N || D.M >= (1ll << 31) ||
+        D.N >= (1ll << 31))
+        return FP8BQ_ERR_SHAPE;
+    *empty = D.batch == 0 || D.M == 0 || D.N == 0;
+    if (*empty) return FP8BQ_OK;
+    if (D.batch > 1 && D.out_batch_stride < 0) return FP8BQ_ERR_SHAPE;
+    if (D.batch > 1 && D.out_batch_stride < (D.M - 1) * D.ld_out + D.N) return FP8BQ_ERR_OVERLAP;
+    if (D.y_u8 == nullptr || D.descale_f32 == nullptr || D.out == nullptr) return FP8BQ_ERR_NULL;
+    if ((uintptr_t)D.descale_f32 % 4 || (uintptr_t)D.out % esize_of(D.dtype_out))
+        return FP8BQ_ERR_ALIGN;
+    return FP8BQ_OK;
+}
+
+bool dequant_vector_ok(const fp8bq_dequant_desc &D) {
+    const int oes = esize_of(D.dtype_out);
+    const int64_t obs = D.batch > 1 ? D.out_batch_stride : 0;
+    return D.N % 16 == 0 && D.block_n % 16 == 0 && (uintptr_t)D.y_u8 % 16 == 0 &&
+           (uintptr_t)D.out % 16 == 0 && (D.ld_out * oes) % 16 == 0 && (obs * oes) % 16 == 0;
+}
+
+template <int MAXD>
+cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<int> &idx,
+                                 bool vector, int oes, cudaStream_t st) {
+    static thread_local DequantPack<MAXD> p;
+    size_t i = 0;
+    while (i < idx.size()) {
+        p.n = 0;
+        p.pad_ = 0;
+        p.total = 0;
+        while (i < idx.size() && p.n < MAXD) {
+            const fp8bq_dequant_desc &D = t[idx[i]];
+            DequantDesc &o = p.d[p.n];
+            o.y = D.y_u8;
+            o.s = D.descale_f32;
+            o.out = D.out;
+            o.M = D.M;
+            o.N = D.N;
+            o.ldo = D.ld_out;
+            o.obs = D.batch > 1 ? D.out_batch_stride : 0;
+            o.bm = D.block_m;
+            o.bn = D.block_n;
+            o.gm = (int32_t)cdiv(D.M, D.block_m);
+            o.gn = (int32_t)cdiv(D.N, D.block_n);
+            o.begin = p.total;
+            o.items = (uint64_t)(D.batch * D.M * D.N) / (vector ? 16u : 1u);
+            p.total += o.items;
+            ++p.n;
+            ++i;
+        }
+        const cudaError_t e = launch_dequant<MAXD>(p, oes, vector, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+fp8bq_status run_dequant(const fp8bq_dequant_desc *t, int n, cudaStream_t stream) {
+    if (n < 0) return FP8BQ_ERR_ARG;
+    if (n > 0 && t == nullptr) return FP8BQ_ERR_NULL;
+    std::vector<char> empty((size_t)n, 0);
+    bool any = false;
+    for (int i = 0; i < n; ++i) {
+        bool e = false;
+        const fp8bq_status st = check_dequant_desc(t[i], &e);
+        if (st != FP8BQ_OK) return st;
+        empty[i] = e;
+        any |= !e;
+    }
+    if (!any) return FP8BQ_OK;
+    // Outputs may overlap nothing; codes and descales are inputs.
+    std::vector<Span> sp;
+    for (int i = 0; i < n; ++i) {
+        if (empty[i]) continue;
+        const fp8bq_dequant_desc &D = t[i];
+        const int64_t oes = esize_of(D.dtype_out), b1 = D.batch - 1;
+        const int64_t gm = cdiv(D.M, D.block_m), gn = cdiv(D.N, D.block_n);
+        const int64_t obs = D.batch > 1 ? D.out_batch_stride : 0;
+        const uintptr_t o = (uintptr_t)D.out, y = (uintptr_t)D.y_u8, s = (uintptr_t)D.descale_f32;
+        sp.push_back({o, o + (uintptr_t)((b1 * obs + (D.M - 1) * D.ld_out + D.N) * oes), true});
+        sp.push_back({y, y + (uintptr_t)(D.batch * D.M * D.N), false});
+        sp.push_back({s, s + (uintptr_t)(D.batch * gm * gn * 4), false});
+    }
+    std::sort(sp.begin(), sp.end(), [](const Span &a, const Span &b) { return a.lo < b.lo; });
+    uintptr_t out_end = 0, in_end = 0;
+    for (const Span &x : sp) {
+        if (x.out) {
+            if (x.lo < out_end || x.lo < in_end) return FP8BQ_ERR_OVERLAP;
+            out_end = std::max(out_end, x.hi);
+        } else {
+            if (x.lo < out_end) return FP8BQ_ERR_OVERLAP;
+            in_end = std::max(in_end, x.hi);
+        }
+    }
+    const fp8bq_status sd = check_device();
+    if (sd != FP8BQ_OK) return sd;
+    const bool generic_only = g_path.load() == FP8BQ_PATH_GENERIC;
+    std::vector<int> groups[2][2];  // [vector][output is bf16]
+    for (int i = 0; i < n; ++i) {
+        if (empty[i]) continue;
+        const bool v = !generic_only && dequant_vector_ok(t[i]);
+        groups[v][t[i].dtype_out == FP8BQ_BF16].push_back(i);
+    }
+    for (int v = 0; v < 2; ++v)
+        for (int b = 0; b < 2; ++b) {
+            const std::vector<int> &g = groups[v][b];
+            if (g.empty()) continue;
+            const cudaError_t e =
+                g.size() <= (size_t)kMaxDescSmall
+                    ? launch_dequant_group<kMaxDescSmall>(t, g, v, b ? 2 : 4, stream)
+                    : launch_dequant_group<kMaxDescLarge>(t, g, v, b ? 2 : 4, stream);
+            if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
+        }
+    return FP8BQ_OK;
+}
+
+// ------------------------------------------------------------------ per-tensor scales
+
+template <int MAXD>
+cudaError_t launch_scale_group(const fp8bq_scale_desc *t, const std::vector<int> &idx, int es,
+                               float *scale_out, cudaStream_t st) {
+    static thread_local ScalePack<MAXD> p;
+    size_t i = 0;
+    while (i < idx.size()) {
+        p.n = 0;
+        p.pad_ = 0;
+        p.total = 0;
+        p.acc = reinterpret_cast<uint32_t *>(scale_out);
+        while (i < idx.size() && p.n < MAXD) {
+            const fp8bq_scale_desc &D = t[idx[i]];
+            ScaleDesc &o = p.d[p.n];
+            o.x = D.x;
+            o.numel = D.numel;
+            o.begin = p.total;
+            o.items = (uint64_t)cdiv(D.numel, kScaleItem);
+            o.out = idx[i];
+            o.pad_ = 0;
+            p.total += o.items;
+            ++p.n;
+            ++i;
+        }
+        if (p.total == 0) continue;
+        const cudaError_t e = launch_scale_amax<MAXD>(p, es, st);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out,
+                              cudaStream_t stream) {
+    if (n < 0) return FP8BQ_ERR_ARG;
+    if (n == 0) return FP8BQ_OK;
+    if (t == nullptr || scale_out == nullptr) return FP8BQ_ERR_NULL;
+    if ((uintptr_t)scale_out % 4) return FP8BQ_ERR_ALIGN;
+    const uintptr_t o_lo = (uintptr_t)scale_out, o_hi = o_lo + (uintptr_t)n * 4;
+    for (int i = 0; i < n; ++i) {
+        const fp8bq_scale_desc &D = t[i];
+        if (D.dtype_in != FP8BQ_BF16 && D.dtype_in != FP8BQ_F32) return FP8BQ_ERR_DTYPE;
+        if (D.numel < 0) return FP8BQ_ERR_SHAPE;
+        if (D.numel == 0) continue;
+        if (D.x == nullptr) return FP8BQ_ERR_NULL;
+        const int es = esize_of(D.dtype_in);
+        if ((uintptr_t)D.x % es) return FP8BQ_ERR_ALIGN;
+        const uintptr_t lo = (uintptr_t)D.x, hi = lo + (uintptr_t)(D.numel * es);
+        if (lo < o_hi && o_lo < hi) return FP8BQ_ERR_OVERLAP;
+    }
+    const fp8bq_status sd = check_device();
+    if (sd != FP8BQ_OK) return sd;
+    if (cudaMemsetAsync(scale_out, 0, (size_t)n * 4, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8BQ_ERR_DEVICE;
+    }
+    std::vector<int> groups[2];  // [is fp32]
+    for (int i = 0; i < n; ++i)
+        if (t[i].numel > 0) groups[t[i].dtype_in == FP8BQ_F32].push_back(i);
+    for (int g = 0; g < 2; ++g) {
+        if (groups[g].empty()) continue;
+        const int es = g ? 4 : 2;
+        const cudaError_t e =
+            groups[g].size() <= (size_t)kMaxDescSmall
+                ? launch_scale_group<kMaxDescSmall>(t, groups[g], es, scale_out, stream)
+                : launch_scale_group<kMaxDescLarge>(t, groups[g], es, scale_out, stream);
+        if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
+    }
+    return launch_scale_finalize(scale_out, n, stream) == cudaSuccess ? FP8BQ_OK
+                                                                       : FP8BQ_ERR_DEVICE;
+}
+
 }  // namespace
 
 extern "C" {
+
+fp8bq_status fp8bq_tensor_scale(const fp8bq_scale_desc *desc_table, int n_tensors,
+                                float *scale_out, cudaStream_t stream) {
+    return run_tensor_scale(desc_table, n_tensors, scale_out, stream);
+}
 
 fp8bq_status fp8bq_quantize(const void *x, fp8bq_dtype dtype_in, int64_t M, int64_t N, int64_t ld,
                             int block_m, int block_n, uint8_t *y_u8, float *descale_f32,
@@ -417,6 +619,31 @@ fp8bq_status fp8bq_quantize(const void *x, fp8bq_dtype dtype_in, int64_t M, int6
 fp8bq_status fp8bq_quantize_batched(const fp8bq_desc *desc_table, int n_tensors,
                                     cudaStream_t stream) {
     return run(desc_table, n_tensors, stream);
+}
+
+fp8bq_status fp8bq_dequantize(const uint8_t *y_u8, const float *descale_f32, int64_t batch,
+                              int64_t M, int64_t N, int block_m, int block_n, void *out,
+                              fp8bq_dtype dtype_out, int64_t ld_out, int64_t out_batch_stride,
+                              cudaStream_t stream) {
+    fp8bq_dequant_desc D;
+    std::memset(&D, 0, sizeof D);
+    D.y_u8 = y_u8;
+    D.descale_f32 = descale_f32;
+    D.out = out;
+    D.batch = batch;
+    D.M = M;
+    D.N = N;
+    D.ld_out = ld_out;
+    D.out_batch_stride = out_batch_stride;
+    D.dtype_out = (int32_t)dtype_out;
+    D.block_m = block_m;
+    D.block_n = block_n;
+    return run_dequant(&D, 1, stream);
+}
+
+fp8bq_status fp8bq_dequantize_batched(const fp8bq_dequant_desc *desc_table, int n_tensors,
+                                      cudaStream_t stream) {
+    return run_dequant(desc_table, n_tensors, stream);
 }
 
 const char *fp8bq_status_string(fp8bq_status s) {

@@ -157,15 +157,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// One probe that may suspend the thread in hardware for up to `hint_ns`
+// (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
+                                                   uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+#ifndef FP8BQ_WAIT_HINT_NS
+#define FP8BQ_WAIT_HINT_NS 0  // 0: the hardware's default suspend time
+#endif
+
 // Wait for a phase, giving up after `limit_ns` of global time or as soon as
 // *abort becomes nonzero.  Returns true if the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns,
                                                   const volatile int *abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto probe = [&]() {
+        return FP8BQ_WAIT_HINT_NS ? mbar_try_wait_hint(bar, parity, FP8BQ_WAIT_HINT_NS)
+                                  : mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (probe()) return true;
         if (abort != nullptr && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }

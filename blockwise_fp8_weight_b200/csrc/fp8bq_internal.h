@@ -57,7 +57,7 @@ static_assert(sizeof(TmaPack<kMaxDescTma>) < 32000, "kernel parameter limit");
 // Kernel variants, by input element size and team shape.
 enum class Variant : int {
     Generic = 0,
-    VecT16 = 1,   // a team of 16 threads per block (blocks of <= 16 vectors)
+    VecT16 = 1,   // a team of 16 threads per 8 stacked blocks of one row-step each
     VecT64 = 2,   // a team of 64 threads per block (<= 512 vectors)
     VecTBig = 3,  // one team per CTA (<= 2048 vectors)
     Tma = 4,
@@ -70,6 +70,57 @@ template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
 cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st);
 
+// Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
+// grouped launch walks the concatenated work items (16 codes per item for the
+// vector kernel, 1 for the generic one) of all descriptors of a pack.
+struct DequantDesc {
+    const uint8_t *y;   // [batch, M, N] codes
+    const float *s;     // [batch, gm, gn] descales
+    void *out;          // matrix b at out + b * obs elements, row stride ldo
+    int64_t M, N, ldo, obs;
+    int32_t bm, bn, gm, gn;
+    uint64_t begin;     // first work item of this descriptor
+    uint64_t items;     // batch * M * N / (16 or 1)
+};
+static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
+
+template <int MAXD>
+struct DequantPack {
+    int32_t n;
+    int32_t pad_;
+    uint64_t total;
+    DequantDesc d[MAXD];
+};
+static_assert(sizeof(DequantPack<kMaxDescLarge>) < 32000, "kernel parameter limit");
+
+template <int MAXD>
+cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st);
+
+// Per-tensor scales (fp8bq_scale.cu): the tensors of a pack are cut into
+// work items of kScaleItem elements; every warp folds its items' absmax into
+// acc[out] (the caller's output, zeroed first, as fp32 bit patterns).
+constexpr int64_t kScaleItem = 4096;
+struct ScaleDesc {
+    const void *x;
+    int64_t numel;
+    uint64_t begin;   // first work item
+    uint64_t items;   // ceil(numel / kScaleItem)
+    int32_t out;      // index into the output
+    int32_t pad_;
+};
+template <int MAXD>
+struct ScalePack {
+    int32_t n;
+    int32_t pad_;
+    uint64_t total;
+    uint32_t *acc;
+    ScaleDesc d[MAXD];
+};
+static_assert(sizeof(ScalePack<kMaxDescLarge>) < 32000, "kernel parameter limit");
+template <int MAXD>
+cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t st);
+cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st);
+
 // Device error word access (fp8bq_kernels.cu).
 cudaError_t read_and_clear_error_word(uint32_t *out);
 
@@ -77,7 +128,9 @@ cudaError_t read_and_clear_error_word(uint32_t *out);
 constexpr int kVecTeamThreads(Variant v, int esize) {
     return v == Variant::VecT16 ? 16 : v == Variant::VecT64 ? 64 : (esize == 2 ? 256 : 512);
 }
-constexpr int kVecSlots(Variant v) { return v == Variant::VecT16 ? 1 : 8; }
+constexpr int kVecSlots(Variant v) { return 8; }
+// Blocks per tile along M: the small-block kernel stacks 8 blocks per tile.
+constexpr int kTileBlocksM(Variant v) { return v == Variant::VecT16 ? 8 : 1; }
 
 constexpr int kTmaConsumerThreads = 256;
 constexpr int kTmaStageBytes = 32768;

@@ -39,7 +39,7 @@ constexpr uint64_t kDrainLimitNs = 2000000000ull;
 #define FP8BQ_VEC_L2_PREFETCH 0   // vector kernel: bulk-prefetch the tile after next into L2
 #endif
 #ifndef FP8BQ_TMA_STAGES_BF16
-#define FP8BQ_TMA_STAGES_BF16 6   // 32 KB ring slots per TMA CTA (bf16 tiles)
+#define FP8BQ_TMA_STAGES_BF16 4   // 32 KB ring slots per TMA CTA (bf16 tiles)
 #endif
 #ifndef FP8BQ_TMA_STAGES_F32
 #define FP8BQ_TMA_STAGES_F32 3    // 64 KB ring slots per TMA CTA (fp32 tiles)
@@ -59,16 +59,20 @@ struct Tile {
     int b, bi, bj;    // coordinates (TMA)
 };
 
-template <int ESIZE, int MAXD>
+// Tile t of a launch.  A tile is G vertically adjacent blocks of one matrix
+// (G = 1 except for the small-block vector kernel); rows counts the valid
+// rows of all G blocks and sdst points at the first block's descale.
+template <int ESIZE, int G = 1, int MAXD>
 __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d) {
     while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
     const TileDesc &D = p.d[d];
     const uint32_t local = t - D.tile_begin;
-    const uint32_t per = (uint32_t)D.gm * (uint32_t)D.gn;
+    const uint32_t gmu = G == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + G - 1) / G;
+    const uint32_t per = gmu * (uint32_t)D.gn;
     const uint32_t b = local / per;
     const uint32_t rem = local - b * per;
-    const uint32_t bi = rem / (uint32_t)D.gn;
-    const uint32_t bj = rem - bi * (uint32_t)D.gn;
+    const uint32_t bi = (rem / (uint32_t)D.gn) * G;
+    const uint32_t bj = rem - (bi / G) * (uint32_t)D.gn;
     const int64_t r0 = (int64_t)bi * D.bm, c0 = (int64_t)bj * D.bn;
     Tile T;
     T.src = (const char *)D.x + ((int64_t)b * D.xbs + r0 * D.ld + c0) * ESIZE;
@@ -76,7 +80,7 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     T.sdst = D.s + (int64_t)b * D.sbs + (int64_t)bi * D.gn + bj;
     T.ld = D.ld;
     T.ldy = D.N;
-    T.rows = (int)min((int64_t)D.bm, (int64_t)D.M - r0);
+    T.rows = (int)min((int64_t)G * D.bm, (int64_t)D.M - r0);
     T.cols = (int)min((int64_t)D.bn, (int64_t)D.N - c0);
     T.b = (int)b;
     T.bi = (int)bi;
@@ -84,24 +88,32 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     return T;
 }
 
-// absmax bits of a 16-byte vector
-template <int ESIZE>
-__device__ __forceinline__ uint32_t vec_absmax(const uint4 &v, uint32_t m) {
-    if constexpr (ESIZE == 2) {
-        m = dev::absmax_bf16x2(m, v.x);
-        m = dev::absmax_bf16x2(m, v.y);
-        m = dev::absmax_bf16x2(m, v.z);
-        m = dev::absmax_bf16x2(m, v.w);
-    } else {
-        m = max(m, v.x & 0x7fffffffu);
-        m = max(m, v.y & 0x7fffffffu);
-        m = max(m, v.z & 0x7fffffffu);
-        m = max(m, v.w & 0x7fffffffu);
+// absmax bits of V 16-byte vectors: four independent running maxima (one per
+// 32-bit lane of the vectors) so the max chains overlap, merged at the end.
+template <int ESIZE, int V>
+__device__ __forceinline__ uint32_t tile_absmax(const uint4 (&R)[V]) {
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        if constexpr (ESIZE == 2) {
+            m0 = dev::absmax_bf16x2(m0, R[i].x);
+            m1 = dev::absmax_bf16x2(m1, R[i].y);
+            m2 = dev::absmax_bf16x2(m2, R[i].z);
+            m3 = dev::absmax_bf16x2(m3, R[i].w);
+        } else {
+            m0 = max(m0, R[i].x & 0x7fffffffu);
+            m1 = max(m1, R[i].y & 0x7fffffffu);
+            m2 = max(m2, R[i].z & 0x7fffffffu);
+            m3 = max(m3, R[i].w & 0x7fffffffu);
+        }
     }
-    return m;
+    if constexpr (ESIZE == 2)
+        return dev::absmax_bf16x2(dev::absmax_bf16x2(m0, m1), dev::absmax_bf16x2(m2, m3));
+    else
+        return max(max(m0, m1), max(m2, m3));
 }
 
-// fp32 bit pattern of the absmax accumulated by vec_absmax
+// fp32 bit pattern of the absmax accumulated by vec_absmax / tile_absmax
 template <int ESIZE>
 __device__ __forceinline__ uint32_t absmax_to_f32_bits(uint32_t m) {
     if constexpr (ESIZE == 2)
@@ -133,9 +145,14 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
 // 16-byte pieces of a row, so each warp load covers whole 256-byte row
 // segments.  bm and bn are the same for every tensor of a launch.
 
-template <int ESIZE, int TEAM, int V, int CTA, int MAXD>
+//
+// G > 1 (small blocks): a tile is G vertically adjacent blocks and slot i of
+// every thread holds a vector of block i (one block is exactly one row-step
+// of the team, bm * vpr == TEAM), so each slot is reduced on its own.
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
+    static_assert(G == 1 || (G == V && TEAM <= 32), "per-slot blocks need a sub-warp team");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -171,16 +188,35 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     auto prefetch = [&](uint32_t tn) {
         if (!FP8BQ_VEC_L2_PREFETCH || tn >= p.total_tiles) return;
         int dd = d;
-        const Tile T = make_tile<ESIZE>(p, tn, dd);
+        const Tile T = make_tile<ESIZE, G>(p, tn, dd);
         for (int r = lane; r < T.rows; r += TEAM)
             dev::prefetch_l2(T.src + (int64_t)r * T.ld * ESIZE, (uint32_t)(T.cols * ESIZE));
     };
 
-    auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
-        uint32_t m = 0;
+    auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
+        const int bm = p.d[0].bm;
 #pragma unroll
-        for (int i = 0; i < V; ++i) m = vec_absmax<ESIZE>(R[i], m);
-        m = absmax_to_f32_bits<ESIZE>(m);
+        for (int i = 0; i < V; ++i) {
+            const uint4 one[1] = {R[i]};
+            uint32_t m = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
+#pragma unroll
+            for (int o = TEAM / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(shfl_mask, m, o));
+            if (i * bm >= T.rows) continue;  // block below the matrix
+            float s, r;
+            dev::block_scale(m, kEps, s, r);
+            const int rr = row0 + i * rstep;
+            if (rr < T.rows && colv < T.cols)
+                vec_quant_store<ESIZE>(R[i], dev::splat2(r), T.dst + (int64_t)rr * T.ldy + colv);
+            if (lane == 0) T.sdst[(int64_t)i * p.d[0].gn] = s;
+        }
+    };
+
+    auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
+        if constexpr (G > 1) {
+            process_slots(R, T);
+            return;
+        }
+        uint32_t m = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE>(R));
         if constexpr (TEAM <= 32) {
 #pragma unroll
             for (int o = TEAM / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(shfl_mask, m, o));
@@ -205,7 +241,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     };
 
     uint4 A[V], B[V];
-    Tile ta = make_tile<ESIZE>(p, t, d);
+    Tile ta = make_tile<ESIZE, G>(p, t, d);
     load(A, ta);
     uint32_t it = 0;
     while (true) {
@@ -213,7 +249,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         const bool h1 = t1 < p.total_tiles;
         Tile tb;
         if (h1) {
-            tb = make_tile<ESIZE>(p, t1, d);
+            tb = make_tile<ESIZE, G>(p, t1, d);
             load(B, tb);
             prefetch(t1 + stride);
         }
@@ -222,7 +258,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         const uint32_t t2 = t1 + stride;
         const bool h2 = t2 < p.total_tiles;
         if (h2) {
-            ta = make_tile<ESIZE>(p, t2, d);
+            ta = make_tile<ESIZE, G>(p, t2, d);
             load(A, ta);
             prefetch(t2 + stride);
         }
@@ -281,6 +317,26 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
     }
 }
 
+// The tiles one TMA CTA processes, in order: every gridDim.x-th tile
+// (strided), or one contiguous run of tiles per CTA.
+#ifndef FP8BQ_TMA_CONTIGUOUS
+#define FP8BQ_TMA_CONTIGUOUS 0
+#endif
+struct TileWalk {
+    uint32_t t, end, step;
+    __device__ __forceinline__ explicit TileWalk(uint32_t total) {
+        if (FP8BQ_TMA_CONTIGUOUS) {
+            t = (uint32_t)((uint64_t)total * blockIdx.x / gridDim.x);
+            end = (uint32_t)((uint64_t)total * (blockIdx.x + 1) / gridDim.x);
+            step = 1;
+        } else {
+            t = blockIdx.x;
+            end = total;
+            step = gridDim.x;
+        }
+    }
+};
+
 // ============================================================== TMA kernel
 //
 // Warp 0 (one elected lane) is the producer: for each tile of this CTA it
@@ -300,6 +356,15 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
     constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
     extern __shared__ __align__(1024) uint8_t ring[];
+    // Where each slot's tile goes: written by the producer before it arms the
+    // slot's barrier, read by the consumers after the barrier completes.
+    struct SlotInfo {
+        uint8_t *dst;
+        float *sdst;
+        int64_t ldy;
+        int32_t rows, cols;
+    };
+    __shared__ SlotInfo info[STAGES];
     __shared__ __align__(8) uint64_t full[STAGES];
     __shared__ __align__(8) uint64_t empty[STAGES];
     __shared__ uint32_t red[2][kTmaConsumerThreads / 32];
@@ -325,7 +390,8 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         int d = 0;
         uint32_t k = 0;
         bool dropped0 = false;
-        for (uint32_t t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++k) {
+        for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
+            const uint32_t t = w.t;
             const int st = (int)(k % STAGES);
             const uint32_t round = k / STAGES;
             if (round > 0 &&
@@ -337,6 +403,11 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                 break;
             }
             const Tile T = make_tile<ESIZE>(p, t, d);
+            info[st].dst = T.dst;
+            info[st].sdst = T.sdst;
+            info[st].ldy = T.ldy;
+            info[st].rows = T.rows;
+            info[st].cols = T.cols;
             dev::mbar_arrive_expect_tx(&full[st], tile_bytes);
             if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
                 dropped0 = true;  // fault injection: this slot's barrier can never complete
@@ -363,13 +434,13 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     const int row0 = ct / vpr;
     const int rstep = kTmaConsumerThreads / vpr;
     const int colv = cv * VEC;
-    int d = 0;
     uint32_t k = 0;
-    for (uint32_t t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++k) {
+    for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
         const int st = (int)(k % STAGES);
         const bool ok = dev::mbar_wait_bounded(&full[st], (k / STAGES) & 1u, p.wait_limit_ns,
                                                &abort_flag);
-        const Tile T = make_tile<ESIZE>(p, t, d);
+        SlotInfo T = {nullptr, nullptr, 0, 0, 0};
+        if (ok) T = info[st];
         uint4 R[V];
         const uint8_t *stage = ring + (size_t)st * STAGE_BYTES;
 #pragma unroll
@@ -383,10 +454,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         __syncwarp();
         if (lane == 0 && ok) dev::mbar_arrive(&empty[st]);
 
-        uint32_t m = 0;
-#pragma unroll
-        for (int i = 0; i < V; ++i) m = vec_absmax<ESIZE>(R[i], m);
-        m = __reduce_max_sync(0xffffffffu, absmax_to_f32_bits<ESIZE>(m));
+        uint32_t m = __reduce_max_sync(0xffffffffu, absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE>(R)));
         if (lane == 0) red[k & 1][cw] = m;
         if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
             if (ct == 0) {
@@ -441,9 +509,9 @@ unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {
     return (unsigned)(need < cap ? (need ? need : 1) : cap);
 }
 
-template <int ESIZE, int TEAM, int V, int CTA, int MAXD>
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
 cudaError_t launch_vector_t(const DescPack<MAXD> &p, cudaStream_t st) {
-    auto kern = k_vector<ESIZE, TEAM, V, CTA, MAXD>;
+    auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD>;
     static int occ = resident_ctas(kern, CTA, 0);
     const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
     kern<<<grid, CTA, 0, st>>>(p);
@@ -456,16 +524,16 @@ template <int MAXD>
 cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st) {
     if (esize == 2) {
         switch (v) {
-            case Variant::VecT16: return launch_vector_t<2, 16, 1, 256, MAXD>(p, st);
-            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, MAXD>(p, st);
-            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, MAXD>(p, st);
+            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(p, st);
+            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(p, st);
+            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(p, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (v) {
-        case Variant::VecT16: return launch_vector_t<4, 16, 1, 256, MAXD>(p, st);
-        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, MAXD>(p, st);
-        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, MAXD>(p, st);
+        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(p, st);
+        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(p, st);
+        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(p, st);
         default: return cudaErrorInvalidValue;
     }
 }

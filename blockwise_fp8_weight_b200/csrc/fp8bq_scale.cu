@@ -1,0 +1,107 @@
+// fp8bq_scale.cu -- per-tensor FP8 scales: scale = max(max|x|, eps) / 448.
+//
+// The FP8-RL report recalibrates the Q/K/V scales of its FP8 KV cache every
+// RL step (abstract).  This is the block recipe of the weight quantizer
+// applied to a whole tensor: a read-only pass (HBM-bound, numel * esize bytes)
+// then one division pair per tensor.
+//
+// Pass 1 (k_scale_amax): the tensors of a launch are cut into items of
+// kScaleItem elements; each CTA walks items grid-stride, each thread folds 16
+// elements into a running max of bit patterns, each warp reduces and does one
+// atomicMax into the output slot, which holds fp32 bit patterns meanwhile
+// (the output was zeroed first; for non-negative floats the integer order of
+// the bits is the numeric order).  Pass 2 (k_scale_finalize) turns the bits
+// into the scale in place.
+#include "fp8bq_device.cuh"
+#include "fp8bq_internal.h"
+
+namespace fp8bq {
+namespace {
+
+template <int ESIZE>
+__device__ __forceinline__ uint32_t elem_abs(const char *base, int64_t i) {
+    if constexpr (ESIZE == 2)
+        return ((uint32_t)__ldg((const unsigned short *)base + i) & 0x7fffu) << 16;
+    else
+        return __float_as_uint(__ldg((const float *)base + i)) & 0x7fffffffu;
+}
+
+template <int ESIZE, int MAXD>
+__global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ ScalePack<MAXD> p) {
+    constexpr int VEC = 16 / ESIZE;            // elements per 16-byte load
+    constexpr int LOADS = 16 / VEC;            // loads per thread per item (16 elements)
+    static_assert(256 * 16 == kScaleItem, "item = 256 threads x 16 elements");
+    int d = 0;
+    for (uint64_t it = blockIdx.x; it < p.total; it += gridDim.x) {
+        while (it >= p.d[d].begin + p.d[d].items) ++d;
+        const ScaleDesc &D = p.d[d];
+        const int64_t e0 = (int64_t)(it - D.begin) * kScaleItem;
+        const int64_t len = min((int64_t)kScaleItem, D.numel - e0);
+        const char *base = (const char *)D.x + e0 * ESIZE;
+        uint32_t m = 0;
+        if (len == kScaleItem && ((uintptr_t)base & 15) == 0) {
+            uint4 v[LOADS];
+#pragma unroll
+            for (int j = 0; j < LOADS; ++j)
+                v[j] = dev::ldg_stream_v4(base + ((int64_t)j * 256 + threadIdx.x) * 16);
+#pragma unroll
+            for (int j = 0; j < LOADS; ++j) {
+                if constexpr (ESIZE == 2) {
+                    m = dev::absmax_bf16x2(m, v[j].x);
+                    m = dev::absmax_bf16x2(m, v[j].y);
+                    m = dev::absmax_bf16x2(m, v[j].z);
+                    m = dev::absmax_bf16x2(m, v[j].w);
+                } else {
+                    m = max(m, max(v[j].x & 0x7fffffffu, v[j].y & 0x7fffffffu));
+                    m = max(m, max(v[j].z & 0x7fffffffu, v[j].w & 0x7fffffffu));
+                }
+            }
+            if constexpr (ESIZE == 2) m = max(m & 0xffffu, m >> 16) << 16;
+        } else {
+            for (int64_t i = threadIdx.x; i < len; i += 256) m = max(m, elem_abs<ESIZE>(base, i));
+        }
+        m = __reduce_max_sync(0xffffffffu, m);
+        if ((threadIdx.x & 31) == 0 && m) atomicMax(p.acc + D.out, m);
+    }
+}
+
+__global__ void k_scale_finalize(float *scale_out, int n) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        const uint32_t bits = reinterpret_cast<const uint32_t *>(scale_out)[i];
+        const float a = fmaxf(__uint_as_float(bits), kEps);
+        scale_out[i] = __fdiv_rn(a, kFp8Max);
+    }
+}
+
+}  // namespace
+
+template <int MAXD>
+cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t st) {
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    const uint64_t cap = (uint64_t)sms * 8;
+    const unsigned grid = (unsigned)(p.total < cap ? (p.total ? p.total : 1) : cap);
+    if (esize == 2)
+        k_scale_amax<2, MAXD><<<grid, 256, 0, st>>>(p);
+    else
+        k_scale_amax<4, MAXD><<<grid, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st) {
+    const int blocks = (n + 255) / 256;
+    k_scale_finalize<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(scale_out, n);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_scale_amax<kMaxDescSmall>(const ScalePack<kMaxDescSmall> &, int,
+                                                      cudaStream_t);
+template cudaError_t launch_scale_amax<kMaxDescLarge>(const ScalePack<kMaxDescLarge> &, int,
+                                                      cudaStream_t);
+
+}  // namespace fp8bq

@@ -138,6 +138,79 @@ typedef struct fp8bq_desc {
 FP8BQ_API fp8bq_status fp8bq_quantize_batched(const fp8bq_desc *desc_table, int n_tensors,
                                     cudaStream_t stream);
 
+/*
+ * Dequantize: the consumer side of the descale ("_scale_inv") tensor
+ * ("vllm_fp8_utils.py" docs, section 3): for every matrix b of a stack,
+ *
+ *     out[b, r, c] = decode(y[b, r, c]) * descale[b, r / block_m, c / block_n]
+ *
+ * with one fp32 multiply rounded to nearest even; for bf16 output that fp32
+ * product is then rounded to bf16 (nearest even).  The pages print no
+ * dequantization code; this is the plain reading of the descale's meaning.
+ *
+ *   y_u8         device, [batch, M, N] contiguous e4m3fn codes (the layout
+ *                fp8bq_quantize writes).
+ *   descale_f32  device, [batch, ceil(M/block_m), ceil(N/block_n)] contiguous.
+ *   out          device, matrix b at out + b * out_batch_stride (elements),
+ *                rows ld_out >= N elements apart, dtype_out bf16 or fp32.
+ *
+ * Codes 0x7F / 0xFF (NaN) are never written by the quantizer and dequantize
+ * to NaN.  Same checks, status codes and stream semantics as fp8bq_quantize.
+ */
+FP8BQ_API fp8bq_status fp8bq_dequantize(const uint8_t *y_u8, const float *descale_f32,
+                                        int64_t batch, int64_t M, int64_t N, int block_m,
+                                        int block_n, void *out, fp8bq_dtype dtype_out,
+                                        int64_t ld_out, int64_t out_batch_stride,
+                                        cudaStream_t stream);
+
+/* One matrix stack of a grouped dequantization (fields as in fp8bq_dequantize). */
+typedef struct fp8bq_dequant_desc {
+    const uint8_t *y_u8;       /* device, [batch, M, N] contiguous codes */
+    const float *descale_f32;  /* device, [batch, ceil(M/bm), ceil(N/bn)] contiguous */
+    void *out;                 /* device, dtype_out elements */
+    int64_t batch, M, N;
+    int64_t ld_out;            /* output row stride, elements, >= N */
+    int64_t out_batch_stride;  /* elements; ignored for batch == 1 */
+    int32_t dtype_out;         /* fp8bq_dtype */
+    int32_t block_m, block_n;
+    int32_t reserved;          /* set to 0 */
+} fp8bq_dequant_desc;
+
+/*
+ * Dequantize a list of matrix stacks in as few launches as possible (one per
+ * kernel variant and output dtype), e.g. every weight of a layer or a model.
+ * desc_table is HOST memory, read during the call only.  All descriptors are
+ * checked before anything is launched.
+ */
+FP8BQ_API fp8bq_status fp8bq_dequantize_batched(const fp8bq_dequant_desc *desc_table,
+                                                int n_tensors, cudaStream_t stream);
+
+/*
+ * Per-tensor FP8 scales, e.g. the Q/K/V scales of an FP8 KV cache, which the
+ * FP8-RL report recalibrates every RL step (its abstract; the pages print no
+ * formula).  Reading: the weight recipe applied to a whole tensor as one
+ * block,
+ *
+ *     scale_out[i] = max(max |x_i|, eps) / 448      (fp32, eps = 1e-10f)
+ *
+ * so x_i / scale_out[i] fits e4m3fn and scale_out[i] is its dequantization
+ * multiplier.  One grouped launch covers all n tensors.
+ *
+ *   desc_table  HOST memory, n_tensors entries: contiguous device tensors of
+ *               numel >= 0 elements (numel 0 gives eps / 448).
+ *   scale_out   device, n_tensors floats, written (used as the accumulator
+ *               while the call runs; it must not overlap any input).
+ */
+typedef struct fp8bq_scale_desc {
+    const void *x;      /* device, numel contiguous elements */
+    int64_t numel;
+    int32_t dtype_in;   /* fp8bq_dtype */
+    int32_t reserved;   /* set to 0 */
+} fp8bq_scale_desc;
+
+FP8BQ_API fp8bq_status fp8bq_tensor_scale(const fp8bq_scale_desc *desc_table, int n_tensors,
+                                          float *scale_out, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
 

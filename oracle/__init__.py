@@ -77,6 +77,13 @@ def lib() -> ctypes.CDLL:
             L.fp8bq_oracle_e4m3_decode_array.restype = None
             L.fp8bq_oracle_dequantize.argtypes = [vp, vp, i64, i64, ctypes.c_int, ctypes.c_int, vp]
             L.fp8bq_oracle_dequantize.restype = None
+            L.fp8bq_oracle_dequantize_bf16.argtypes = [vp, vp, i64, i64, ctypes.c_int,
+                                                       ctypes.c_int, vp]
+            L.fp8bq_oracle_dequantize_bf16.restype = None
+            L.fp8bq_oracle_tensor_scale.argtypes = [vp, ctypes.c_int, i64, f32]
+            L.fp8bq_oracle_tensor_scale.restype = f32
+            L.fp8bq_oracle_bf16.argtypes = [f32]
+            L.fp8bq_oracle_bf16.restype = ctypes.c_uint16
             _lib = L
     return _lib
 
@@ -156,11 +163,28 @@ def quantize_block(x: np.ndarray, M: int, N: int, ld: int | None, bm: int, bn: i
     return y, float(s[0])
 
 
-def dequantize(y: np.ndarray, s: np.ndarray, bm: int, bn: int) -> np.ndarray:
-    """x_hat = dec(y) * s per block, fp32."""
+def dequantize(y: np.ndarray, s: np.ndarray, bm: int, bn: int, out_dtype: str = "f32"):
+    """x_hat = dec(y) * s per block: one fp32 multiply; ``out_dtype`` "f32"
+    returns float32, "bf16" returns uint16 bf16 bits (the fp32 product
+    rounded to nearest even)."""
     y = np.ascontiguousarray(y, dtype=np.uint8)
     s = np.ascontiguousarray(s, dtype=np.float32)
     M, N = y.shape
-    out = np.empty((M, N), dtype=np.float32)
-    lib().fp8bq_oracle_dequantize(_ptr(y), _ptr(s), M, N, bm, bn, _ptr(out))
+    gm, gn = grid_shape(M, N, bm, bn)
+    if s.size < gm * gn:
+        raise ValueError("descale grid too small")
+    if out_dtype == "f32":
+        out = np.empty((M, N), dtype=np.float32)
+        lib().fp8bq_oracle_dequantize(_ptr(y), _ptr(s), M, N, bm, bn, _ptr(out))
+    elif out_dtype == "bf16":
+        out = np.empty((M, N), dtype=np.uint16)
+        lib().fp8bq_oracle_dequantize_bf16(_ptr(y), _ptr(s), M, N, bm, bn, _ptr(out))
+    else:
+        raise ValueError(out_dtype)
     return out
+
+
+def tensor_scale(x: np.ndarray, eps: float = EPS) -> np.float32:
+    """Per-tensor scale max(max|x|, eps) / 448 of a whole array (bf16 bits or fp32)."""
+    x = np.ascontiguousarray(x)
+    return np.float32(lib().fp8bq_oracle_tensor_scale(_ptr(x), _dtype_code(x), x.size, float(eps)))

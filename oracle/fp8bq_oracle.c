@@ -28,6 +28,9 @@
  *   [K4] same page, "背景知识": the format is float8_e4m3fn.
  *   [U3] "vllm_fp8_utils.py" docs, section 3 "权重量化": the descale is emitted
  *        as "<name>_scale_inv" next to the fp8 weight.
+ *   [P1] "FP8-RL: A Practical and Stable Low-Precision Stack for LLM
+ *        Reinforcement Learning", abstract: the KV cache is also FP8, with its
+ *        Q/K/V scales recalibrated every RL step.
  *
  * Readings taken where the pages are silent (each is listed in the design
  * notes):
@@ -233,7 +236,13 @@ void fp8bq_oracle_e4m3_decode_array(const uint8_t *q, int64_t n, float *out)
         out[i] = fp8bq_oracle_e4m3_decode(q[i]);
 }
 
-/* Dequantize x_hat[r, c] = dec(y[r, c]) * s[r / bm, c / bn] ([U3]). */
+/*
+ * Dequantization, the consumer side of the "_scale_inv" tensor ([U3]): the
+ * descale is the multiplier that maps codes back to weights,
+ *     x_hat[r, c] = dec(y[r, c]) * s[r / bm, c / bn]
+ * with one fp32 multiply (round to nearest even).  The pages print no
+ * dequantization code; this is the plain reading of the descale's meaning.
+ */
 void fp8bq_oracle_dequantize(const uint8_t *y, const float *s, int64_t M, int64_t N,
                              int bm, int bn, float *out)
 {
@@ -241,4 +250,46 @@ void fp8bq_oracle_dequantize(const uint8_t *y, const float *s, int64_t M, int64_
     for (int64_t r = 0; r < M; ++r)
         for (int64_t c = 0; c < N; ++c)
             out[r * N + c] = fp8bq_oracle_e4m3_decode(y[r * N + c]) * s[(r / bm) * gn + c / bn];
+}
+
+/* fp32 -> bf16 bits, round to nearest, ties to even (finite inputs). */
+uint16_t fp8bq_oracle_bf16(float v)
+{
+    uint32_t b = bits_from_f32(v);
+    uint32_t keep = b >> 16, rest = b & 0xffffu;
+    if (rest > 0x8000u || (rest == 0x8000u && (keep & 1u)))
+        keep += 1; /* a carry into the exponent is the correct rounding */
+    return (uint16_t)keep;
+}
+
+/* Dequantization to bf16: the fp32 product above, rounded to bf16. */
+void fp8bq_oracle_dequantize_bf16(const uint8_t *y, const float *s, int64_t M, int64_t N,
+                                  int bm, int bn, uint16_t *out)
+{
+    int64_t gn = (N + bn - 1) / bn;
+    for (int64_t r = 0; r < M; ++r)
+        for (int64_t c = 0; c < N; ++c)
+            out[r * N + c] = fp8bq_oracle_bf16(fp8bq_oracle_e4m3_decode(y[r * N + c]) *
+                                               s[(r / bm) * gn + c / bn]);
+}
+
+/*
+ * Per-tensor scale of the FP8 KV cache, recalibrated each step ([P1]): the
+ * pages name the recalibration but print no formula; the reading is the
+ * weight recipe ([K2]) applied to the whole tensor as one block,
+ *     s = max(max |x|, eps) / 448
+ * (fp32, round to nearest).  x holds numel contiguous elements.
+ */
+float fp8bq_oracle_tensor_scale(const void *x, int dtype, int64_t numel, float eps)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < numel; ++i) {
+        float ax = load_elem(x, dtype, 0, 0, i);
+        ax = ax < 0.0f ? -ax : ax;
+        if (ax > amax)
+            amax = ax;
+    }
+    if (amax < eps)
+        amax = eps;
+    return amax / E4M3_MAX;
 }

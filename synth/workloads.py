@@ -118,6 +118,16 @@ def edge() -> list[TensorSpec]:
     return out
 
 
+def qkv_activations(tokens: int = 16384) -> list[TensorSpec]:
+    """Q, K, V activations of one Qwen3-8B-shaped attention layer for a batch of
+    `tokens` tokens (Q: 32 heads x 128, K and V: 8 KV heads x 128), bf16,
+    N(0,1) x per-token lognormal(0,1): the inputs of the per-step KV-cache
+    scale recalibration."""
+    return [TensorSpec(f"act.{name}", tokens, width, seed=4, tensor_id=i, sigma=1.0,
+                       row_lognormal_sigma=1.0)
+            for i, (name, width) in enumerate((("q", 4096), ("k", 1024), ("v", 1024)))]
+
+
 def materialize(spec: TensorSpec, nthreads: int | None = None) -> np.ndarray:
     """Host array for ``spec`` (flat, numel_storage elements)."""
     if spec.meta.get("recipe") == "small":

@@ -146,7 +146,7 @@ def test_variant_choice(path_guard):
     assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_AUTO
     assert P(desc()) == fq.FP8BQ_PATH_TMA                          # 128x128, aligned
     assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR   # 256-B blocks
-    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_TMA      # 8 KB blocks
+    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_VECTOR   # 8 KB blocks
     assert P(desc(batch=1, block_m=32, block_n=64)) == fq.FP8BQ_PATH_VECTOR   # 4 KB blocks
     assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_VECTOR) == fq.FP8BQ_OK
@@ -178,3 +178,89 @@ def test_debug_knobs():
 @pytest.mark.skipif(not NO_GPU, reason="checks the no-device path")
 def test_sync_status_without_device():
     assert fq.fp8bq_sync_status(0) == fq.FP8BQ_ERR_DEVICE
+
+
+def dq(**kw):
+    a = dict(y_u8=Y, descale_f32=S, batch=1, M=256, N=384, block_m=128, block_n=128, out=X,
+             dtype_out=fq.FP8BQ_BF16, ld_out=384, out_batch_stride=0, stream=0)
+    a.update(kw)
+    return fq.fp8bq_dequantize(**a)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dtype_out=3), fq.FP8BQ_ERR_DTYPE),
+    (dict(block_m=0), fq.FP8BQ_ERR_BLOCK),
+    (dict(block_m=512, block_n=512), fq.FP8BQ_ERR_BLOCK),
+    (dict(M=-2), fq.FP8BQ_ERR_SHAPE),
+    (dict(ld_out=100), fq.FP8BQ_ERR_SHAPE),
+    (dict(batch=-1), fq.FP8BQ_ERR_SHAPE),
+    (dict(batch=2, out_batch_stride=-1), fq.FP8BQ_ERR_SHAPE),
+    (dict(batch=2, out_batch_stride=256 * 384 - 1), fq.FP8BQ_ERR_OVERLAP),
+    (dict(y_u8=0), fq.FP8BQ_ERR_NULL),
+    (dict(out=0), fq.FP8BQ_ERR_NULL),
+    (dict(out=X + 1), fq.FP8BQ_ERR_ALIGN),
+    (dict(dtype_out=fq.FP8BQ_F32, out=X + 2), fq.FP8BQ_ERR_ALIGN),
+    (dict(descale_f32=S + 1), fq.FP8BQ_ERR_ALIGN),
+    (dict(out=Y - 100), fq.FP8BQ_ERR_OVERLAP),
+    (dict(out=S), fq.FP8BQ_ERR_OVERLAP),
+])
+def test_dequantize_argument_errors(kw, status):
+    assert dq(**kw) == status
+
+
+def test_dequantize_empty_and_no_device():
+    assert dq(M=0, y_u8=0, out=0, descale_f32=0) == fq.FP8BQ_OK
+    assert dq(batch=0) == fq.FP8BQ_OK
+    if NO_GPU:
+        assert dq() == fq.FP8BQ_ERR_DEVICE
+
+
+def ddesc(**kw):
+    d = fq.fp8bq_dequant_desc()
+    a = dict(y_u8=Y, descale_f32=S, out=X, batch=1, M=256, N=384, ld_out=384, out_batch_stride=0,
+             dtype_out=fq.FP8BQ_BF16, block_m=128, block_n=128, reserved=0)
+    a.update(kw)
+    for k, v in a.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_dequantize_batched_layout_and_errors():
+    assert ctypes.sizeof(fq.fp8bq_dequant_desc) == 80
+    B = fq.fp8bq_dequantize_batched
+    assert B([]) == fq.FP8BQ_OK
+    assert B([ddesc()], n_tensors=-1) == fq.FP8BQ_ERR_ARG
+    assert B([ddesc(), ddesc(dtype_out=7, out=X + (1 << 36))]) == fq.FP8BQ_ERR_DTYPE
+    # two descriptors writing the same output
+    assert B([ddesc(), ddesc(y_u8=Y + (1 << 36), descale_f32=S + (1 << 36))]) == \
+        fq.FP8BQ_ERR_OVERLAP
+    # second descriptor's output runs over the first one's codes
+    assert B([ddesc(), ddesc(out=Y, y_u8=Y + (1 << 36), descale_f32=S + (1 << 36))]) == \
+        fq.FP8BQ_ERR_OVERLAP
+    if NO_GPU:
+        assert B([ddesc(), ddesc(out=X + (1 << 36))]) == fq.FP8BQ_ERR_DEVICE
+
+
+def sdesc(**kw):
+    d = fq.fp8bq_scale_desc()
+    a = dict(x=X, numel=4096, dtype_in=fq.FP8BQ_BF16, reserved=0)
+    a.update(kw)
+    for k, v in a.items():
+        setattr(d, k, v)
+    return d
+
+
+def test_tensor_scale_argument_errors():
+    T = lambda descs, out=S, n=None: fq.fp8bq_tensor_scale(descs, out, n_tensors=n)  # noqa: E731
+    assert ctypes.sizeof(fq.fp8bq_scale_desc) == 24
+    assert T([sdesc()], n=-1) == fq.FP8BQ_ERR_ARG
+    assert T([], n=0) == fq.FP8BQ_OK
+    assert T([sdesc()], out=0) == fq.FP8BQ_ERR_NULL
+    assert T([sdesc()], out=S + 2) == fq.FP8BQ_ERR_ALIGN
+    assert T([sdesc(dtype_in=5)]) == fq.FP8BQ_ERR_DTYPE
+    assert T([sdesc(numel=-1)]) == fq.FP8BQ_ERR_SHAPE
+    assert T([sdesc(x=0)]) == fq.FP8BQ_ERR_NULL
+    assert T([sdesc(x=X + 1)]) == fq.FP8BQ_ERR_ALIGN
+    assert T([sdesc(x=S - 100)]) == fq.FP8BQ_ERR_OVERLAP
+    if NO_GPU:
+        assert T([sdesc(), sdesc(x=0, numel=0)]) == fq.FP8BQ_ERR_DEVICE

@@ -395,3 +395,84 @@ def test_golden_order_case_discriminates():
     assert via_rcp == int(case["y"][1], 16)
     assert via_div == int(case["y_if_divided_directly"][1], 16)
     assert via_rcp != via_div
+
+
+# ------------------------------------------------------- dequantization
+
+
+def test_bf16_rounding_matches_library_cast():
+    rng = np.random.default_rng(17)
+    pats = rng.integers(0, 2**32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    v = pats.view(np.float32)
+    v = v[np.isfinite(v) & (np.abs(v) < 3.0e38)]
+    got = np.array([oracle.lib().fp8bq_oracle_bf16(float(x)) for x in v[:20000]], dtype=np.uint16)
+    want = v[:20000].astype(ml_dtypes.bfloat16).view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_dequantize_is_one_rounded_product(random_cases):
+    """x_hat = RN_f32(dec(q) * s) exactly; the bf16 output is that value
+    rounded to bf16 (nearest even), checked in exact rational arithmetic."""
+    from tests.exact import round_bf16
+    rng = np.random.default_rng(23)
+    for sp, x in random_cases:
+        y, s = oracle.quantize(x, sp.M, sp.N)
+        xf = oracle.dequantize(y, s, 128, 128, "f32")
+        xb = oracle.dequantize(y, s, 128, 128, "bf16")
+        d = oracle.e4m3_decode(y)
+        for k in rng.integers(0, y.size, size=400):
+            r, c = divmod(int(k), sp.N)
+            prod = round_f32(frac(d[r, c]) * frac(s[r // 128, c // 128]))
+            assert frac(xf[r, c]) == prod
+            assert frac(bf16_bits_to_f32(xb[r, c])) == round_bf16(prod)
+
+
+def test_dequantize_roundtrip_on_grid():
+    """Scale 1 (absmax exactly 448): dequantization returns the grid value of
+    each code, so every on-grid input comes back exactly."""
+    x, q = _grid_block("f32", np.random.default_rng(4))
+    y, s = oracle.quantize(x, 128, 128)
+    assert s[0, 0] == 1.0
+    back = oracle.dequantize(y, s, 128, 128).ravel()
+    g = H.grid()
+    want = np.where(q & 0x80, -g[q & 0x7F], g[q & 0x7F]).astype(np.float32)
+    assert np.array_equal(back, want)
+    on = np.isin(np.abs(x).astype(np.float64), g)
+    assert on.sum() > 10000 and np.array_equal(back[on], x[on])
+
+
+def test_dequantize_error_bound(random_cases):
+    """|x_hat - x| <= s * ulp_e4m3(x * r) / 2 + one fp32 rounding of each side."""
+    for sp, x in random_cases:
+        y, s = oracle.quantize(x, sp.M, sp.N)
+        xf = as_f32(x).reshape(sp.M, sp.N).astype(np.float64)
+        back = oracle.dequantize(y, s, 128, 128).astype(np.float64)
+        ss = np.repeat(np.repeat(s.astype(np.float64), 128, 0), 128, 1)[:sp.M, :sp.N]
+        r = np.repeat(np.repeat((np.float32(1) / s).astype(np.float64), 128, 0), 128, 1)[:sp.M, :sp.N]
+        v = np.clip(xf * r, -448, 448)
+        bound = ss * _ulp_e4m3(v.astype(np.float32)) / 2 + (np.abs(xf) + np.abs(back)) * 2.0**-22
+        assert (np.abs(back - xf) <= bound).all()
+
+
+# ------------------------------------------------------- per-tensor scale
+
+
+def test_tensor_scale_closed_forms():
+    """max(max|x|, eps)/448 in exact arithmetic; eps floor on zeros; invariant
+    under negation and permutation; equal to the block recipe's descale when
+    the tensor is a single block."""
+    rng = np.random.default_rng(31)
+    for sp in [TensorSpec("t1", 64, 4096, seed=91, tensor_id=1, sigma=1.0, row_lognormal_sigma=1.0),
+               TensorSpec("t2", 33, 1000, dtype="f32", seed=91, tensor_id=2, dist=DIST_STUDENT_T3)]:
+        x = W.materialize(sp)
+        s = oracle.tensor_scale(x)
+        a = max(Fraction(float(np.abs(as_f32(x)).max())), frac(EPS))
+        assert frac(s) == round_f32(a / 448)
+        assert oracle.tensor_scale(x[rng.permutation(x.size)]) == s
+        neg = x ^ np.uint16(0x8000) if x.dtype == np.uint16 else -x
+        assert oracle.tensor_scale(neg) == s
+        y, sb = oracle.quantize(x, 1, x.size, bm=1, bn=x.size)
+        assert sb[0, 0] == s
+    z = np.zeros(1000, dtype=np.uint16)
+    assert frac(oracle.tensor_scale(z)) == round_f32(frac(EPS) / 448)
+    assert oracle.tensor_scale(np.array([448.0, -1.0], dtype=np.float32)) == 1.0
