@@ -145,28 +145,59 @@ Variant vector_variant(const fp8bq_desc &D) {
     return Variant::Generic;
 }
 
-bool tma_fits(const fp8bq_desc &D) {
+// Geometry of the TMA kernel for a tensor: a ring slot (one tile) holds
+// `group` vertically stacked blocks, at most 256 rows and 128x128 elements;
+// consumer thread ct holds rows ct / vpr + i * rs (rs = 256 / vpr).  Either
+// a block is a whole number of row-steps (reduced across the CTA) or it is
+// a power-of-two group of at most 32 lanes within one row-step (reduced with
+// shuffles, `subwarp`).  Returns false if neither holds.
+bool tma_geom(const fp8bq_desc &D, int *group, bool *subwarp) {
     const int es = esize_of(D.dtype_in), vec = 16 / es;
-    if (D.block_m > 256 || D.block_n > 256 || (D.block_n * es) % 16) return false;
-    if ((int64_t)D.block_m * D.block_n * es > 128 * 128 * es) return false;
+    if (D.block_n > 256 || (D.block_n * es) % 16) return false;
     const int vpr = D.block_n / vec;
     if (!is_pow2(vpr) || vpr > kTmaConsumerThreads) return false;
-    const int64_t slots = 128 * 128 * es / 16 / kTmaConsumerThreads;
-    if (cdiv(D.block_m, kTmaConsumerThreads / vpr) > slots) return false;
+    const int rs = kTmaConsumerThreads / vpr;
+    const int slots = 128 * 128 * es / 16 / kTmaConsumerThreads;
+    const int max_rows = std::min(256, 128 * 128 / D.block_n);
+    if (D.block_m > max_rows) return false;
     if (D.batch > 1 && D.x_batch_stride == 0) return false;
-    return vector_aligned(D);
+    if (!vector_aligned(D)) return false;
+    if (D.block_m % rs == 0) {
+        const int spb = D.block_m / rs;
+        if (spb > slots) return false;
+        *group = std::min(max_rows / D.block_m, slots / spb);
+        *subwarp = false;
+        return *group >= 1;
+    }
+    const int64_t lanes = (int64_t)D.block_m * vpr;
+    if (lanes <= 32 && is_pow2(lanes) && rs % D.block_m == 0) {
+        *group = max_rows / D.block_m;
+        *subwarp = true;
+        return *group >= 1;
+    }
+    return false;
 }
 
-// AUTO: the TMA ring for blocks of at least 32 KB (one ring slot holds one
-// block, so smaller blocks leave too few bytes in flight), the register-tile
-// vector kernel for smaller aligned blocks, the generic kernel otherwise.
-constexpr int64_t kTmaMinBlockBytes = 32768;
+bool tma_fits(const fp8bq_desc &D) {
+    int g;
+    bool sub;
+    return tma_geom(D, &g, &sub);
+}
+
+// AUTO: the TMA ring when one block fills a ring slot of at least 16 KB
+// (measured: with stacked small blocks the ring's 8 consumer warps spend too
+// long per tile, and the register-tile vector kernel is 2-2.5x faster), the
+// vector kernel for other aligned tensors, the generic kernel otherwise.
+constexpr int64_t kTmaMinSlotBytes = 16384;
 
 Variant choose(const fp8bq_desc &D, int path) {
     if (path == FP8BQ_PATH_GENERIC) return Variant::Generic;
-    if (path == FP8BQ_PATH_TMA && tma_fits(D)) return Variant::Tma;
-    if (path == FP8BQ_PATH_AUTO && tma_fits(D) &&
-        (int64_t)D.block_m * D.block_n * esize_of(D.dtype_in) >= kTmaMinBlockBytes)
+    int g;
+    bool sub;
+    const bool tma = tma_geom(D, &g, &sub);
+    if (path == FP8BQ_PATH_TMA && tma) return Variant::Tma;
+    if (path == FP8BQ_PATH_AUTO && tma && g == 1 &&
+        (int64_t)D.block_m * D.block_n * esize_of(D.dtype_in) >= kTmaMinSlotBytes)
         return Variant::Tma;
     if (!vector_aligned(D)) return Variant::Generic;
     return vector_variant(D);
@@ -238,7 +269,10 @@ bool encode_map(const fp8bq_desc &D, CUtensorMap *out) {
     const int es = esize_of(D.dtype_in);
     cuuint64_t dims[3] = {(cuuint64_t)D.N, (cuuint64_t)D.M, (cuuint64_t)D.batch};
     cuuint64_t strides[2] = {(cuuint64_t)(D.ld * es), (cuuint64_t)(key.xbs * es)};
-    cuuint32_t box[3] = {(cuuint32_t)D.block_n, (cuuint32_t)D.block_m, 1};
+    int group = 1;
+    bool sub = false;
+    if (!tma_geom(D, &group, &sub)) return false;
+    cuuint32_t box[3] = {(cuuint32_t)D.block_n, (cuuint32_t)(group * D.block_m), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUtensorMap m;
     CUresult r = fn(&m,
@@ -257,8 +291,19 @@ bool encode_map(const fp8bq_desc &D, CUtensorMap *out) {
 
 // ------------------------------------------------------------------ launches
 
+// Blocks stacked along M in one tile of variant v.
+int tile_group(const fp8bq_desc &D, Variant v) {
+    if (v == Variant::Tma) {
+        int g = 1;
+        bool sub = false;
+        tma_geom(D, &g, &sub);
+        return g;
+    }
+    return kTileBlocksM(v);
+}
+
 uint64_t tiles_of(const fp8bq_desc &D, Variant v) {
-    return (uint64_t)D.batch * cdiv(cdiv(D.M, D.block_m), kTileBlocksM(v)) * cdiv(D.N, D.block_n);
+    return (uint64_t)D.batch * cdiv(cdiv(D.M, D.block_m), tile_group(D, v)) * cdiv(D.N, D.block_n);
 }
 
 void fill_tile_desc(const fp8bq_desc &D, Variant v, uint32_t begin, TileDesc *o) {
@@ -284,7 +329,7 @@ void pack_header(DescPack<MAXD> &p) {
     p.n = 0;
     p.total_tiles = 0;
     p.inject = g_inject.load();
-    p.pad_ = 0;
+    p.group = 1;
     p.wait_limit_ns = g_wait_limit_ns.load();
 }
 
@@ -329,7 +374,11 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
             ++P.p.n;
             ++i;
         }
-        const cudaError_t e = launch_tma(es, P, st);
+        int group = 1;
+        bool sub = false;
+        tma_geom(t[idx[0]], &group, &sub);  // the same for every tensor of the group
+        P.p.group = group;
+        const cudaError_t e = launch_tma(es, sub, P, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -447,7 +496,9 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.gm = (int32_t)cdiv(D.M, D.block_m);
             o.gn = (int32_t)cdiv(D.N, D.block_n);
             o.begin = p.total;
-            o.items = (uint64_t)(D.batch * D.M * D.N) / (vector ? 16u : 1u);
+            // vector: warp items of 32 x 16 codes per row; generic: one element
+            o.items = vector ? (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32)
+                             : (uint64_t)(D.batch * D.M * D.N);
             p.total += o.items;
             ++p.n;
             ++i;

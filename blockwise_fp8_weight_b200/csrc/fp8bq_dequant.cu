@@ -47,26 +47,33 @@ __device__ __forceinline__ const DequantDesc &find(const DequantPack<MAXD> &p, u
     return p.d[d];
 }
 
-// 16 codes per work item (one 16-byte load), all in one block (N and block_n
-// are multiples of 16).
+// Vector kernel: a work item is a warp-wide row segment of 32 x 16 codes
+// (one 16-byte load per lane; N and block_n are multiples of 16, so the 16
+// codes of a lane share one descale).  Items are numbered row-major over
+// (matrix, row, segment) and walked grid-stride by warps, so index
+// arithmetic is paid once per 512 codes.
 template <int OES, int MAXD>
 __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ DequantPack<MAXD> p) {
+    const int lane = threadIdx.x & 31;
+    const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
     int d = 0;
-    for (uint64_t k = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; k < p.total;
-         k += (uint64_t)gridDim.x * blockDim.x) {
+    for (uint64_t k = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < p.total;
+         k += warps) {
         const DequantDesc &a = find(p, k, d);
         const int64_t n16 = a.N / 16;
-        const int64_t per_b = a.M * n16;
+        const int64_t segs = (n16 + 31) / 32;
         const int64_t local = (int64_t)(k - a.begin);
-        const int64_t b = local / per_b;
-        const int64_t rem = local - b * per_b;
-        const int64_t r = rem / n16;
-        const int64_t c = (rem - r * n16) * 16;
+        const int64_t row_all = local / segs;            // b * M + r
+        const int64_t chunk = (local - row_all * segs) * 32 + lane;
+        if (chunk >= n16) continue;
+        const int64_t b = row_all / a.M;
+        const int64_t r = row_all - b * a.M;
+        const int64_t c = chunk * 16;
         const float s = __ldg(a.s + (b * a.gm + r / a.bm) * a.gn + c / a.bn);
         uint64_t ss;
         asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
         uint4 q;
-        const uint8_t *src = a.y + (b * a.M + r) * a.N + c;
+        const uint8_t *src = a.y + row_all * a.N + c;
         asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
                      : "=r"(q.x), "=r"(q.y), "=r"(q.z), "=r"(q.w)
                      : "l"(src));
@@ -143,7 +150,7 @@ unsigned dq_grid(uint64_t work) {
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st) {
-    const unsigned grid = dq_grid(p.total);
+    const unsigned grid = dq_grid(vector ? p.total * 32 : p.total);  // vector: a warp per item
     if (vector) {
         if (out_esize == 2)
             k_dequant_vec<2, MAXD><<<grid, 256, 0, st>>>(p);

@@ -37,7 +37,7 @@ struct DescPack {
     int32_t n;              // descriptors used
     uint32_t total_tiles;   // sum of tiles
     uint32_t inject;        // FP8BQ_INJECT_* flags (TMA kernel)
-    uint32_t pad_;
+    int32_t group;          // blocks stacked along M per TMA tile (TMA kernel)
     uint64_t wait_limit_ns; // bound of every device wait (TMA kernel)
     TileDesc d[MAXD];
 };
@@ -68,11 +68,12 @@ template <int MAXD>
 cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st);
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
-cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st);
+cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<kMaxDescTma> &p, cudaStream_t st);
 
 // Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
-// grouped launch walks the concatenated work items (16 codes per item for the
-// vector kernel, 1 for the generic one) of all descriptors of a pack.
+// grouped launch walks the concatenated work items (a warp-wide row segment
+// of 32 x 16 codes for the vector kernel, one element for the generic one) of
+// all descriptors of a pack.
 struct DequantDesc {
     const uint8_t *y;   // [batch, M, N] codes
     const float *s;     // [batch, gm, gn] descales
@@ -80,7 +81,7 @@ struct DequantDesc {
     int64_t M, N, ldo, obs;
     int32_t bm, bn, gm, gn;
     uint64_t begin;     // first work item of this descriptor
-    uint64_t items;     // batch * M * N / (16 or 1)
+    uint64_t items;     // work items of this descriptor
 };
 static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
 
@@ -99,7 +100,7 @@ cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vecto
 // Per-tensor scales (fp8bq_scale.cu): the tensors of a pack are cut into
 // work items of kScaleItem elements; every warp folds its items' absmax into
 // acc[out] (the caller's output, zeroed first, as fp32 bit patterns).
-constexpr int64_t kScaleItem = 4096;
+constexpr int64_t kScaleItem = 8192;
 struct ScaleDesc {
     const void *x;
     int64_t numel;

@@ -63,16 +63,20 @@ struct Tile {
 // (G = 1 except for the small-block vector kernel); rows counts the valid
 // rows of all G blocks and sdst points at the first block's descale.
 template <int ESIZE, int G = 1, int MAXD>
-__device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d) {
+__device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d,
+                                          int g_rt = 1) {
     while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
     const TileDesc &D = p.d[d];
     const uint32_t local = t - D.tile_begin;
-    const uint32_t gmu = G == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + G - 1) / G;
+    // G is the compile-time group; g_rt a run-time one (used when G == 0)
+    const uint32_t grp = G == 0 ? (uint32_t)g_rt : (uint32_t)G;
+    const uint32_t gmu = grp == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + grp - 1) / grp;
     const uint32_t per = gmu * (uint32_t)D.gn;
     const uint32_t b = local / per;
     const uint32_t rem = local - b * per;
-    const uint32_t bi = (rem / (uint32_t)D.gn) * G;
-    const uint32_t bj = rem - (bi / G) * (uint32_t)D.gn;
+    const uint32_t bgi = rem / (uint32_t)D.gn;
+    const uint32_t bi = bgi * grp;
+    const uint32_t bj = rem - bgi * (uint32_t)D.gn;
     const int64_t r0 = (int64_t)bi * D.bm, c0 = (int64_t)bj * D.bn;
     Tile T;
     T.src = (const char *)D.x + ((int64_t)b * D.xbs + r0 * D.ld + c0) * ESIZE;
@@ -80,7 +84,7 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     T.sdst = D.s + (int64_t)b * D.sbs + (int64_t)bi * D.gn + bj;
     T.ld = D.ld;
     T.ldy = D.N;
-    T.rows = (int)min((int64_t)G * D.bm, (int64_t)D.M - r0);
+    T.rows = (int)min((int64_t)grp * D.bm, (int64_t)D.M - r0);
     T.cols = (int)min((int64_t)D.bn, (int64_t)D.N - c0);
     T.b = (int)b;
     T.bi = (int)bi;
@@ -120,6 +124,27 @@ __device__ __forceinline__ uint32_t absmax_to_f32_bits(uint32_t m) {
         return max(m & 0xffffu, m >> 16) << 16;
     else
         return m;
+}
+
+// Scales of V blocks whose absmax bits m[0..V-1] every lane of an aligned
+// group of L >= V lanes already holds: lane q of the group computes block q
+// (one division pair per lane instead of V), then every lane fetches the V
+// reciprocals by shuffle.  Returns the scale of block (lane % L) (valid for
+// lanes with lane % L < V, which write the descales).
+template <int V>
+__device__ __forceinline__ float group_scales(const uint32_t (&m)[V], int L, uint32_t mask,
+                                              float (&r)[V]) {
+    const int lane = threadIdx.x & 31;
+    const int q = lane & (L - 1);
+    uint32_t mq = m[0];
+#pragma unroll
+    for (int i = 1; i < V; ++i) mq = (q == i) ? m[i] : mq;
+    float sq, rq;
+    dev::block_scale(mq, kEps, sq, rq);
+    const int base = lane & ~(L - 1);
+#pragma unroll
+    for (int i = 0; i < V; ++i) r[i] = __shfl_sync(mask, rq, base + i);
+    return sq;
 }
 
 // Quantize one 16-byte vector with rr = {r, r} and store its codes (8 bytes
@@ -195,20 +220,24 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
 
     auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
         const int bm = p.d[0].bm;
+        uint32_t m[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const uint4 one[1] = {R[i]};
-            uint32_t m = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
+            m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
 #pragma unroll
-            for (int o = TEAM / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(shfl_mask, m, o));
-            if (i * bm >= T.rows) continue;  // block below the matrix
-            float s, r;
-            dev::block_scale(m, kEps, s, r);
+            for (int o = TEAM / 2; o > 0; o >>= 1) m[i] = max(m[i], __shfl_xor_sync(shfl_mask, m[i], o));
+        }
+        float r[V];
+        const float s_mine = group_scales<V>(m, TEAM, shfl_mask, r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            if (i * bm >= T.rows) break;  // blocks below the matrix
             const int rr = row0 + i * rstep;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], dev::splat2(r), T.dst + (int64_t)rr * T.ldy + colv);
-            if (lane == 0) T.sdst[(int64_t)i * p.d[0].gn] = s;
+                vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv);
         }
+        if (lane < V && lane * bm < T.rows) T.sdst[(int64_t)lane * p.d[0].gn] = s_mine;
     };
 
     auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
@@ -343,18 +372,30 @@ struct TileWalk {
 // waits until the ring slot is free, arms the slot's "full" barrier with the
 // tile's byte count and issues one 3-D tensor-map load (no multicast).  Warps
 // 1..8 are consumers: they wait for "full", copy the tile from shared memory
-// into registers, release the slot ("empty"), reduce the absmax across the 8
-// warps, and quantize + store from registers.  Every wait is bounded; a wait
-// that runs out sets the device error word, all consumers leave together
-// (the reduction barrier also ORs a failure flag), and the producer waits
-// (bounded) for each copy it issued before it returns.
+// into registers, release the slot ("empty"), reduce the absmax, and quantize
+// + store from registers.  Every wait is bounded; a wait that runs out sets
+// the device error word, all consumers leave together (a barrier that also
+// ORs a failure flag), and the producer waits (bounded) for each copy it
+// issued before it returns.
+//
+// A tile is G vertically stacked blocks (one ring slot of up to 32 KB of bf16
+// / 64 KB of fp32; G = 1 for 128x128 blocks).  Consumer thread ct holds the
+// 16-byte vectors (row0 + i * RS, cv), i < V, of the tile, RS = 256 / vpr.
+//   MODE_ONE  (G = 1): the tile is one block, reduced across the 8 consumer
+//             warps (the 128x128 case).
+//   MODE_CTA  (bm a multiple of RS, G > 1): slot i belongs to block
+//             i / (bm / RS); each block is reduced across the 8 warps.
+//   MODE_SUB  (a block is L = bm * vpr <= 32 lanes of one slot): each slot is
+//             reduced within its group of L lanes with shuffles.
+enum { MODE_ONE = 0, MODE_SUB = 1, MODE_CTA = 2 };
 
-template <int ESIZE, int STAGES>
+template <int ESIZE, int STAGES, int MODE>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
     k_tma(const __grid_constant__ TmaPack<kMaxDescTma> P) {
     constexpr int VEC = 16 / ESIZE;
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
     constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
+    constexpr int NW = kTmaConsumerThreads / 32;
     extern __shared__ __align__(1024) uint8_t ring[];
     // Where each slot's tile goes: written by the producer before it arms the
     // slot's barrier, read by the consumers after the barrier completes.
@@ -362,12 +403,12 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         uint8_t *dst;
         float *sdst;
         int64_t ldy;
-        int32_t rows, cols;
+        int32_t rows, cols, gn, pad;
     };
     __shared__ SlotInfo info[STAGES];
     __shared__ __align__(8) uint64_t full[STAGES];
     __shared__ __align__(8) uint64_t empty[STAGES];
-    __shared__ uint32_t red[2][kTmaConsumerThreads / 32];
+    __shared__ uint32_t red[2][V][NW];
     __shared__ volatile int abort_flag;
 
     const DescPack<kMaxDescTma> &p = P.p;
@@ -375,15 +416,15 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             dev::mbar_init(&full[s], 1);
-            dev::mbar_init(&empty[s], kTmaConsumerThreads / 32);
+            dev::mbar_init(&empty[s], NW);
         }
         abort_flag = 0;
         dev::fence_mbar_init();
     }
     __syncthreads();
 
-    const int bm = p.d[0].bm, bn = p.d[0].bn;
-    const uint32_t tile_bytes = (uint32_t)(bm * bn * ESIZE);
+    const int bm = p.d[0].bm, bn = p.d[0].bn, grp = p.group;
+    const uint32_t tile_bytes = (uint32_t)(grp * bm * bn * ESIZE);
 
     if (warp == 0) {
         if (lane != 0) return;
@@ -391,7 +432,6 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         uint32_t k = 0;
         bool dropped0 = false;
         for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
-            const uint32_t t = w.t;
             const int st = (int)(k % STAGES);
             const uint32_t round = k / STAGES;
             if (round > 0 &&
@@ -402,12 +442,13 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                 }
                 break;
             }
-            const Tile T = make_tile<ESIZE>(p, t, d);
+            const Tile T = make_tile<ESIZE, 0>(p, w.t, d, grp);
             info[st].dst = T.dst;
             info[st].sdst = T.sdst;
             info[st].ldy = T.ldy;
             info[st].rows = T.rows;
             info[st].cols = T.cols;
+            info[st].gn = p.d[d].gn;
             dev::mbar_arrive_expect_tx(&full[st], tile_bytes);
             if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
                 dropped0 = true;  // fault injection: this slot's barrier can never complete
@@ -434,19 +475,25 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     const int row0 = ct / vpr;
     const int rstep = kTmaConsumerThreads / vpr;
     const int colv = cv * VEC;
+    const int box_rows = grp * bm;
+    // MODE_CTA: slots per block; MODE_SUB: lanes per block
+    const int spb = MODE == MODE_SUB ? 1 : bm / rstep;
+    const int L = MODE == MODE_SUB ? bm * vpr : 32;
+    const uint32_t sub_mask =
+        L >= 32 ? 0xffffffffu : (((1u << L) - 1u) << (lane & ~(L - 1)));
     uint32_t k = 0;
     for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
         const int st = (int)(k % STAGES);
         const bool ok = dev::mbar_wait_bounded(&full[st], (k / STAGES) & 1u, p.wait_limit_ns,
                                                &abort_flag);
-        SlotInfo T = {nullptr, nullptr, 0, 0, 0};
+        SlotInfo T = {nullptr, nullptr, 0, 0, 0, 0, 0};
         if (ok) T = info[st];
         uint4 R[V];
         const uint8_t *stage = ring + (size_t)st * STAGE_BYTES;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int r = row0 + i * rstep;
-            if (ok && r < bm)
+            if (ok && r < box_rows)
                 R[i] = *reinterpret_cast<const uint4 *>(stage + ((size_t)r * bn + colv) * ESIZE);
             else
                 R[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -454,28 +501,104 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         __syncwarp();
         if (lane == 0 && ok) dev::mbar_arrive(&empty[st]);
 
-        uint32_t m = __reduce_max_sync(0xffffffffu, absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE>(R)));
-        if (lane == 0) red[k & 1][cw] = m;
-        if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
-            if (ct == 0) {
-                atomicOr(&g_error_word, 1u);
-                abort_flag = 1;
+        if constexpr (MODE != MODE_SUB) {
+            if (MODE == MODE_ONE) {  // one block per tile: one CTA-wide reduction
+                uint32_t m = __reduce_max_sync(0xffffffffu,
+                                               absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE>(R)));
+                if (lane == 0) red[k & 1][0][cw] = m;
+            } else {  // per-slot warp maxima; a block's slots are combined below
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const uint4 one[1] = {R[i]};
+                    const uint32_t m = __reduce_max_sync(
+                        0xffffffffu, absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one)));
+                    if (lane == 0) red[k & 1][i][cw] = m;
+                }
             }
-            break;
-        }
-        m = red[k & 1][0];
+            if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
+                if (ct == 0) {
+                    atomicOr(&g_error_word, 1u);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            if (MODE == MODE_ONE) {
+                uint32_t m = red[k & 1][0][0];
 #pragma unroll
-        for (int w = 1; w < kTmaConsumerThreads / 32; ++w) m = max(m, red[k & 1][w]);
-        float s, r;
-        dev::block_scale(m, kEps, s, r);
-        const uint64_t r2 = dev::splat2(r);
+                for (int ww = 1; ww < NW; ++ww) m = max(m, red[k & 1][0][ww]);
+                float s, r;
+                dev::block_scale(m, kEps, s, r);
+                const uint64_t r2 = dev::splat2(r);
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int rr = row0 + i * rstep;
-            if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+                for (int i = 0; i < V; ++i) {
+                    const int rr = row0 + i * rstep;
+                    if (rr < T.rows && colv < T.cols)
+                        vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+                }
+                if (ct == 0) *T.sdst = s;
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int j = i / spb;  // block of slot i
+                    if (j >= grp || j * bm >= T.rows) continue;
+                    uint32_t m = 0;
+                    for (int i2 = j * spb; i2 < (j + 1) * spb; ++i2)
+                        for (int ww = 0; ww < NW; ++ww) m = max(m, red[k & 1][i2][ww]);
+                    float s, r;
+                    dev::block_scale(m, kEps, s, r);
+                    const int rr = row0 + i * rstep;
+                    if (rr < T.rows && colv < T.cols)
+                        vec_quant_store<ESIZE>(R[i], dev::splat2(r),
+                                               T.dst + (int64_t)rr * T.ldy + colv);
+                    if (ct == 0 && i == j * spb) T.sdst[(int64_t)j * T.gn] = s;
+                }
+            }
+        } else {
+            if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
+                if (ct == 0) {
+                    atomicOr(&g_error_word, 1u);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            uint32_t m[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const uint4 one[1] = {R[i]};
+                m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
+                for (int o = L / 2; o > 0; o >>= 1)
+                    m[i] = max(m[i], __shfl_xor_sync(sub_mask, m[i], o));
+            }
+            if (L >= V) {  // one division pair per lane, reciprocals by shuffle
+                float r[V];
+                const float s_mine = group_scales<V>(m, L, sub_mask, r);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int rr = row0 + i * rstep;
+                    if (rr < T.rows && colv < T.cols)
+                        vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]),
+                                               T.dst + (int64_t)rr * T.ldy + colv);
+                }
+                const int q = ct & (L - 1);  // this lane's block: slot q of its group
+                if (q < V) {
+                    const int blk = (row0 + q * rstep) / bm;
+                    if (blk * bm < T.rows) T.sdst[(int64_t)blk * T.gn] = s_mine;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int rr = row0 + i * rstep;
+                    const int blk = rr / bm;
+                    if (blk * bm >= T.rows) continue;  // block below the matrix
+                    float s, r;
+                    dev::block_scale(m[i], kEps, s, r);
+                    if (rr < T.rows && colv < T.cols)
+                        vec_quant_store<ESIZE>(R[i], dev::splat2(r),
+                                               T.dst + (int64_t)rr * T.ldy + colv);
+                    if ((ct & (L - 1)) == 0) T.sdst[(int64_t)blk * T.gn] = s;
+                }
+            }
         }
-        if (ct == 0) *T.sdst = s;
     }
 }
 
@@ -551,10 +674,10 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
 }
 
 namespace {
-template <int ESIZE, int STAGES>
+template <int ESIZE, int STAGES, int MODE>
 cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
     constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
-    auto kern = k_tma<ESIZE, STAGES>;
+    auto kern = k_tma<ESIZE, STAGES, MODE>;
     static cudaError_t attr =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
@@ -564,9 +687,18 @@ cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
 }
 }  // namespace
 
-cudaError_t launch_tma(int esize, const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
-    return esize == 2 ? launch_tma_t<2, FP8BQ_TMA_STAGES_BF16>(p, st)
-                      : launch_tma_t<4, FP8BQ_TMA_STAGES_F32>(p, st);
+cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
+    const int mode = subwarp ? MODE_SUB : p.p.group == 1 ? MODE_ONE : MODE_CTA;
+    if (esize == 2) {
+        constexpr int S = FP8BQ_TMA_STAGES_BF16;
+        return mode == MODE_ONE   ? launch_tma_t<2, S, MODE_ONE>(p, st)
+               : mode == MODE_SUB ? launch_tma_t<2, S, MODE_SUB>(p, st)
+                                  : launch_tma_t<2, S, MODE_CTA>(p, st);
+    }
+    constexpr int S = FP8BQ_TMA_STAGES_F32;
+    return mode == MODE_ONE   ? launch_tma_t<4, S, MODE_ONE>(p, st)
+           : mode == MODE_SUB ? launch_tma_t<4, S, MODE_SUB>(p, st)
+                              : launch_tma_t<4, S, MODE_CTA>(p, st);
 }
 
 cudaError_t read_and_clear_error_word(uint32_t *out) {

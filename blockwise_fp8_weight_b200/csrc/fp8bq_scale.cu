@@ -6,12 +6,13 @@
 // then one division pair per tensor.
 //
 // Pass 1 (k_scale_amax): the tensors of a launch are cut into items of
-// kScaleItem elements; each CTA walks items grid-stride, each thread folds 16
-// elements into a running max of bit patterns, each warp reduces and does one
-// atomicMax into the output slot, which holds fp32 bit patterns meanwhile
-// (the output was zeroed first; for non-negative floats the integer order of
-// the bits is the numeric order).  Pass 2 (k_scale_finalize) turns the bits
-// into the scale in place.
+// kScaleItem elements; each CTA walks items grid-stride and its threads fold
+// them into a running max of bit patterns; when the CTA moves on to another
+// tensor (and at the end) it reduces and does one atomicMax into that
+// tensor's output slot, which holds fp32 bit patterns meanwhile (the output
+// was zeroed first; for non-negative floats the integer order of the bits is
+// the numeric order).  Pass 2 (k_scale_finalize) turns the bits into the
+// scale in place.
 #include "fp8bq_device.cuh"
 #include "fp8bq_internal.h"
 
@@ -26,19 +27,39 @@ __device__ __forceinline__ uint32_t elem_abs(const char *base, int64_t i) {
         return __float_as_uint(__ldg((const float *)base + i)) & 0x7fffffffu;
 }
 
+// Fold a running max into the output slot of tensor `out`: CTA-wide reduce,
+// then one atomicMax (called when a CTA moves to another tensor and at the
+// end, so a tensor sees about one atomic per CTA).
+__device__ __forceinline__ void flush_max(uint32_t m, uint32_t *acc, int out, uint32_t *red) {
+    m = __reduce_max_sync(0xffffffffu, m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = red[0];
+        for (int w = 1; w < 8; ++w) t = max(t, red[w]);
+        if (t) atomicMax(acc + out, t);
+    }
+    __syncthreads();
+}
+
 template <int ESIZE, int MAXD>
 __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ ScalePack<MAXD> p) {
     constexpr int VEC = 16 / ESIZE;            // elements per 16-byte load
-    constexpr int LOADS = 16 / VEC;            // loads per thread per item (16 elements)
-    static_assert(256 * 16 == kScaleItem, "item = 256 threads x 16 elements");
-    int d = 0;
+    constexpr int LOADS = kScaleItem / 256 / VEC;
+    __shared__ uint32_t red[8];
+    int d = 0, cur = -1;
+    uint32_t m = 0;
     for (uint64_t it = blockIdx.x; it < p.total; it += gridDim.x) {
         while (it >= p.d[d].begin + p.d[d].items) ++d;
+        if (d != cur) {  // uniform across the CTA: `it` is per CTA
+            if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red);
+            m = 0;
+            cur = d;
+        }
         const ScaleDesc &D = p.d[d];
         const int64_t e0 = (int64_t)(it - D.begin) * kScaleItem;
         const int64_t len = min((int64_t)kScaleItem, D.numel - e0);
         const char *base = (const char *)D.x + e0 * ESIZE;
-        uint32_t m = 0;
         if (len == kScaleItem && ((uintptr_t)base & 15) == 0) {
             uint4 v[LOADS];
 #pragma unroll
@@ -47,22 +68,20 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
 #pragma unroll
             for (int j = 0; j < LOADS; ++j) {
                 if constexpr (ESIZE == 2) {
-                    m = dev::absmax_bf16x2(m, v[j].x);
-                    m = dev::absmax_bf16x2(m, v[j].y);
-                    m = dev::absmax_bf16x2(m, v[j].z);
-                    m = dev::absmax_bf16x2(m, v[j].w);
+                    const uint32_t a = dev::absmax_bf16x2(dev::absmax_bf16x2(0u, v[j].x), v[j].y);
+                    const uint32_t b = dev::absmax_bf16x2(dev::absmax_bf16x2(0u, v[j].z), v[j].w);
+                    const uint32_t c = dev::absmax_bf16x2(a, b);
+                    m = max(m, max(c & 0xffffu, c >> 16) << 16);
                 } else {
                     m = max(m, max(v[j].x & 0x7fffffffu, v[j].y & 0x7fffffffu));
                     m = max(m, max(v[j].z & 0x7fffffffu, v[j].w & 0x7fffffffu));
                 }
             }
-            if constexpr (ESIZE == 2) m = max(m & 0xffffu, m >> 16) << 16;
         } else {
             for (int64_t i = threadIdx.x; i < len; i += 256) m = max(m, elem_abs<ESIZE>(base, i));
         }
-        m = __reduce_max_sync(0xffffffffu, m);
-        if ((threadIdx.x & 31) == 0 && m) atomicMax(p.acc + D.out, m);
     }
+    if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red);
 }
 
 __global__ void k_scale_finalize(float *scale_out, int n) {

@@ -145,9 +145,10 @@ def test_variant_choice(path_guard):
     P = fq.fp8bq_path_for
     assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_AUTO
     assert P(desc()) == fq.FP8BQ_PATH_TMA                          # 128x128, aligned
-    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR   # 256-B blocks
-    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_VECTOR   # 8 KB blocks
-    assert P(desc(batch=1, block_m=32, block_n=64)) == fq.FP8BQ_PATH_VECTOR   # 4 KB blocks
+    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_VECTOR  # small blocks
+    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(batch=1, block_m=32, block_n=16)) == fq.FP8BQ_PATH_VECTOR  # no TMA geometry
+    assert P(desc(batch=1, block_m=1, block_n=16)) == fq.FP8BQ_PATH_VECTOR   # 8 KB slots
     assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_VECTOR) == fq.FP8BQ_OK
     assert P(desc()) == fq.FP8BQ_PATH_VECTOR
@@ -162,6 +163,8 @@ def test_variant_choice(path_guard):
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_TMA) == fq.FP8BQ_OK
     assert P(desc()) == fq.FP8BQ_PATH_TMA
     assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
+    assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_TMA    # stacked blocks
+    assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_TMA
     assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_GENERIC) == fq.FP8BQ_OK
     assert P(desc()) == fq.FP8BQ_PATH_GENERIC
