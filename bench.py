@@ -48,8 +48,9 @@ if ROOT not in sys.path:
 METRIC = "blockwise FP8 quant GB/s (bytes in+out) and % of B200 HBM peak, 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["blockwise_fp8_weight_b200/csrc/fp8bq_kernels.cu",
-                  "blockwise_fp8_weight_b200/csrc/fp8bq_device.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+                  "blockwise_fp8_weight_b200/csrc/fp8bq_device.cuh",
+                  "blockwise_fp8_weight_b200/csrc/fp8bq_internal.h"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")
 PATHS = {"auto": 0, "vector": 1, "tma": 2, "generic": 3}
 
 
@@ -116,6 +117,9 @@ def workload(name: str):
     if name == "qkv":
         return W.qkv_activations(), ("Q/K/V activations of one Qwen3-8B-shaped attention layer, "
                                      "16384 tokens, bf16 (per-tensor scale recalibration)")
+    if name == "ragged":
+        sp = [t for t in W.edge() if t.name == "edge.bf16.4000x4100"]
+        return sp, "bf16 4000x4100 (rows only 8-byte aligned), block 128x128, Student-t(3) x 0.02"
     if name in ("act_1x128", "blk_64x64"):
         sp = [t for t in W.edge() if t.name.endswith("b1x128" if name == "act_1x128" else "b64x64")]
         return sp, f"bf16 16384x4096, N(0,1) x row lognormal(0,1), blocks {sp[0].block}"
@@ -270,17 +274,20 @@ def kernel_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def traffic_for(workload_name: str, path: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
+def traffic_for(workload_name: str, path: str, launches: int):
+    """DRAM bytes per launch, from the committed ncu record of this workload
+    (profiles/traffic.txt: "<workload> <path> <kernel sources sha256/16>
+    <dram bytes per step>"), if it was taken on the current kernel sources;
+    else None."""
     try:
-        rec = json.load(open(TRAFFIC_FILE))
-    except Exception:
+        lines = open(TRAFFIC_FILE).read().splitlines()
+    except OSError:
         return None
-    for r in rec.get("records", []):
-        if (r.get("workload") == workload_name and r.get("path") == path
-                and r.get("kernel_sources_sha256_16") == kernel_digest()):
-            return r.get("dram_bytes_per_launch")
+    for line in lines:
+        f = line.split()
+        if len(f) == 4 and not line.startswith("#") and f[0] == workload_name and f[1] == path \
+                and f[2] == kernel_digest():
+            return float(f[3]) / max(launches, 1)
     return None
 
 
@@ -543,7 +550,7 @@ def run_ours(args) -> None:
     l2_mb = torch.cuda.get_device_properties(dev).L2_cache_size / 1e6
     launch_s = float(np.mean(step_s)) / max(launches, 1)
     achieved = bytes_per_step / max(launches, 1) / launch_s / 1e9
-    traffic = traffic_for(args.workload, args.path)
+    traffic = traffic_for(args.workload, args.path, launches)
 
     if rank == 0:
         line = {
@@ -719,7 +726,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_model",
                     choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small",
-                             "act_1x128", "blk_64x64", "qkv"])
+                             "act_1x128", "blk_64x64", "qkv", "ragged"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale"],

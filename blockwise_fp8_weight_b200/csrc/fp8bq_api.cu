@@ -178,12 +178,6 @@ bool tma_geom(const fp8bq_desc &D, int *group, bool *subwarp) {
     return false;
 }
 
-bool tma_fits(const fp8bq_desc &D) {
-    int g;
-    bool sub;
-    return tma_geom(D, &g, &sub);
-}
-
 // AUTO: the TMA ring when one block fills a ring slot of at least 16 KB
 // (measured: with stacked small blocks the ring's 8 consumer warps spend too
 // long per tile, and the register-tile vector kernel is 2-2.5x faster), the
