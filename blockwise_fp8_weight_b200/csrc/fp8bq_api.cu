@@ -415,7 +415,10 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         Variant v = choose(D, path);
         CUtensorMap m;
         if (v == Variant::Tma && !encode_map(D, &m)) v = choose(D, FP8BQ_PATH_VECTOR);
-        GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? 0 : D.block_m,
+        // vector / TMA launches need one block shape; generic ones only one
+        // size class (CTA per block for >= 2048 elements, else warp per block)
+        const bool big = (int64_t)D.block_m * D.block_n >= 2048;
+        GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? (int)big : D.block_m,
                    v == Variant::Generic ? 0 : D.block_n};
         size_t g = 0;
         while (g < keys.size() && !(keys[g] == k)) ++g;

@@ -329,6 +329,7 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
         uint32_t m = 0;
         for (int r = 0; r < T.rows; ++r) {
             const char *row = T.src + (int64_t)r * T.ld * ESIZE;
+#pragma unroll 4
             for (int c = lane; c < T.cols; c += 32) m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
         }
         m = __reduce_max_sync(0xffffffffu, m);
@@ -337,12 +338,51 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
         for (int r = 0; r < T.rows; ++r) {
             const char *row = T.src + (int64_t)r * T.ld * ESIZE;
             uint8_t *out = T.dst + (int64_t)r * T.ldy;
+#pragma unroll 4
             for (int c = lane; c < T.cols; c += 32) {
                 const float v = __fmul_rn(elem_f32<ESIZE>(row + c * ESIZE), rc);
                 out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
             }
         }
         if (lane == 0) *T.sdst = s;
+    }
+}
+
+// The same with the whole CTA on one block (blocks of >= 2048 elements): the
+// 8 warps take alternate rows, so a block's loads are spread over 256
+// threads instead of 32.
+template <int ESIZE, int MAXD>
+__global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ DescPack<MAXD> p) {
+    __shared__ uint32_t red[8];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int d = 0;
+    for (uint32_t t = blockIdx.x; t < p.total_tiles; t += gridDim.x) {
+        const Tile T = make_tile<ESIZE>(p, t, d);
+        uint32_t m = 0;
+        for (int r = warp; r < T.rows; r += 8) {
+            const char *row = T.src + (int64_t)r * T.ld * ESIZE;
+#pragma unroll 4
+            for (int c = lane; c < T.cols; c += 32) m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
+        }
+        m = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) red[warp] = m;
+        __syncthreads();
+        m = red[0];
+#pragma unroll
+        for (int w = 1; w < 8; ++w) m = max(m, red[w]);
+        __syncthreads();  // red is rewritten by the next tile
+        float s, rc;
+        dev::block_scale(m, kEps, s, rc);
+        for (int r = warp; r < T.rows; r += 8) {
+            const char *row = T.src + (int64_t)r * T.ld * ESIZE;
+            uint8_t *out = T.dst + (int64_t)r * T.ldy;
+#pragma unroll 4
+            for (int c = lane; c < T.cols; c += 32) {
+                const float v = __fmul_rn(elem_f32<ESIZE>(row + c * ESIZE), rc);
+                out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
+            }
+        }
+        if (threadIdx.x == 0) *T.sdst = s;
     }
 }
 
@@ -663,12 +703,25 @@ cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStr
 
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) {
+    // blocks of >= 2048 elements take one CTA each (the host groups generic
+    // tensors by this size class, so it is uniform per launch)
+    const bool cta = (int64_t)p.d[0].bm * p.d[0].bn >= 2048;
     if (esize == 2) {
-        static int occ = resident_ctas(k_generic<2, MAXD>, 256, 0);
-        k_generic<2, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+        if (cta) {
+            static int occ = resident_ctas(k_generic_cta<2, MAXD>, 256, 0);
+            k_generic_cta<2, MAXD><<<grid_for(p.total_tiles, 1, occ), 256, 0, st>>>(p);
+        } else {
+            static int occ = resident_ctas(k_generic<2, MAXD>, 256, 0);
+            k_generic<2, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+        }
     } else {
-        static int occ = resident_ctas(k_generic<4, MAXD>, 256, 0);
-        k_generic<4, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+        if (cta) {
+            static int occ = resident_ctas(k_generic_cta<4, MAXD>, 256, 0);
+            k_generic_cta<4, MAXD><<<grid_for(p.total_tiles, 1, occ), 256, 0, st>>>(p);
+        } else {
+            static int occ = resident_ctas(k_generic<4, MAXD>, 256, 0);
+            k_generic<4, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+        }
     }
     return cudaGetLastError();
 }
