@@ -422,15 +422,26 @@ def run_ours(args) -> None:
     table = build_descs(specs, lay, x_dev.data_ptr(), y_dev.data_ptr(), s_dev.data_ptr())
     n = len(table)
     assert fq.fp8bq_set_path(PATHS[args.path]) == fq.FP8BQ_OK
-    launches = count_launches(table)
     L = fq.lib()
     stream = torch.cuda.current_stream(dev)
     sh = ctypes.c_void_p(stream.cuda_stream)
+    # grouped: the whole list in one call; per_layer: one call per layer;
+    # per_tensor: one call per tensor (the pages' quant_weights loop)
+    if args.mode == "grouped":
+        calls = [table]
+    elif args.mode == "per_layer":
+        calls = [build_descs(specs, lay, x_dev.data_ptr(), y_dev.data_ptr(), s_dev.data_ptr(), g)
+                 for g in layers_of(specs)]
+    else:
+        calls = [build_descs(specs, lay, x_dev.data_ptr(), y_dev.data_ptr(), s_dev.data_ptr(), [i])
+                 for i in range(len(specs))]
+    launches = sum(count_launches(c) for c in calls)
 
     def step():
-        st = L.fp8bq_quantize_batched(table, n, sh)
-        if st != 0:
-            raise RuntimeError(fq.fp8bq_status_string(st))
+        for c in calls:
+            st = L.fp8bq_quantize_batched(c, len(c), sh)
+            if st != 0:
+                raise RuntimeError(fq.fp8bq_status_string(st))
 
     for _ in range(args.warmup):
         step()
@@ -561,7 +572,8 @@ def run_ours(args) -> None:
             "config": {"workload": wl_desc, "name": args.workload, "tensors": len(specs),
                        "elements": elements, "bytes_per_step": bytes_per_step,
                        "block": list(specs[0].block), "input_dtype": "bf16", "output_dtype": "e4m3fn",
-                       "path": args.path, "parallelism": f"replicas x{world}",
+                       "path": args.path, "calls_per_step": args.mode,
+                       "parallelism": f"replicas x{world}",
                        "l2": (f"no flush: {lay.x_bytes / 1e6:.0f} MB of inputs per step vs "
                               f"{l2_mb:.0f} MB L2") if lay.x_bytes > 2 * l2_mb * 1e6
                        else "inputs fit in L2: latency-bound case",
@@ -729,6 +741,9 @@ def main() -> None:
                              "act_1x128", "blk_64x64", "qkv", "ragged"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",
+                    help="C-ABI calls per step: one grouped call, one per layer, or one per "
+                         "tensor")
     ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale"],
                     default="quantize",
                     help="dequantize: time the reverse map on the quantized workload; "

@@ -68,7 +68,10 @@ template <int MAXD>
 cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st);
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
-cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<kMaxDescTma> &p, cudaStream_t st);
+template <int MAXD>
+cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<MAXD> &p, cudaStream_t st);
+template <int MAXD>
+cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st);
 
 // Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
 // grouped launch walks the concatenated work items (a warp-wide row segment

@@ -62,21 +62,23 @@ struct Tile {
 // Tile t of a launch.  A tile is G vertically adjacent blocks of one matrix
 // (G = 1 except for the small-block vector kernel); rows counts the valid
 // rows of all G blocks and sdst points at the first block's descale.
-template <int ESIZE, int G = 1, int MAXD>
+template <int ESIZE, int G = 1, int MAXD, int H = 1>
 __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d,
                                           int g_rt = 1) {
     while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
     const TileDesc &D = p.d[d];
     const uint32_t local = t - D.tile_begin;
-    // G is the compile-time group; g_rt a run-time one (used when G == 0)
+    // G is the compile-time group; g_rt a run-time one (used when G == 0);
+    // H blocks side by side along N (the paired TMA kernel)
     const uint32_t grp = G == 0 ? (uint32_t)g_rt : (uint32_t)G;
     const uint32_t gmu = grp == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + grp - 1) / grp;
-    const uint32_t per = gmu * (uint32_t)D.gn;
+    const uint32_t gnu = H == 1 ? (uint32_t)D.gn : ((uint32_t)D.gn + H - 1) / H;
+    const uint32_t per = gmu * gnu;
     const uint32_t b = local / per;
     const uint32_t rem = local - b * per;
-    const uint32_t bgi = rem / (uint32_t)D.gn;
+    const uint32_t bgi = rem / gnu;
     const uint32_t bi = bgi * grp;
-    const uint32_t bj = rem - bgi * (uint32_t)D.gn;
+    const uint32_t bj = (rem - bgi * gnu) * H;
     const int64_t r0 = (int64_t)bi * D.bm, c0 = (int64_t)bj * D.bn;
     Tile T;
     T.src = (const char *)D.x + ((int64_t)b * D.xbs + r0 * D.ld + c0) * ESIZE;
@@ -85,7 +87,7 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     T.ld = D.ld;
     T.ldy = D.N;
     T.rows = (int)min((int64_t)grp * D.bm, (int64_t)D.M - r0);
-    T.cols = (int)min((int64_t)D.bn, (int64_t)D.N - c0);
+    T.cols = (int)min((int64_t)H * D.bn, (int64_t)D.N - c0);
     T.b = (int)b;
     T.bi = (int)bi;
     T.bj = (int)bj;
@@ -429,9 +431,9 @@ struct TileWalk {
 //             reduced within its group of L lanes with shuffles.
 enum { MODE_ONE = 0, MODE_SUB = 1, MODE_CTA = 2 };
 
-template <int ESIZE, int STAGES, int MODE>
+template <int ESIZE, int STAGES, int MODE, int MAXD>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
-    k_tma(const __grid_constant__ TmaPack<kMaxDescTma> P) {
+    k_tma(const __grid_constant__ TmaPack<MAXD> P) {
     constexpr int VEC = 16 / ESIZE;
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
     constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
@@ -451,7 +453,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     __shared__ uint32_t red[2][V][NW];
     __shared__ volatile int abort_flag;
 
-    const DescPack<kMaxDescTma> &p = P.p;
+    const DescPack<MAXD> &p = P.p;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -642,6 +644,144 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
     }
 }
 
+// ============================================================== paired TMA kernel
+//
+// The 128x128 bf16 case with two horizontally adjacent blocks per ring slot
+// (box {256, 128}: each row of the tile is 512 contiguous bytes, half the TMA
+// issues and barrier round trips per byte).  Consumer lane l of a warp holds
+// columns of block (l / 16); each block is reduced over its 16 lanes of all 8
+// warps.  Same bounded waits, failure handling and drain as k_tma.
+#ifndef FP8BQ_TMA_PAIR_STAGES
+#define FP8BQ_TMA_PAIR_STAGES 2   // 64 KB ring slots (3 measured 12 % slower)
+#endif
+
+template <int STAGES, int MAXD>
+__global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
+    k_tma_pair(const __grid_constant__ TmaPack<MAXD> P) {
+    constexpr int ESIZE = 2, VEC = 8, BN = 128, BM = 128;
+    constexpr int COLS = 2 * BN;                           // tile columns
+    constexpr int STAGE_BYTES = BM * COLS * ESIZE;         // 64 KB
+    constexpr int VPR = COLS / VEC;                        // 32 vectors per row
+    constexpr int RSTEP = kTmaConsumerThreads / VPR;       // 8 rows per step
+    constexpr int V = BM / RSTEP;                          // 16 vectors per thread
+    constexpr int NW = kTmaConsumerThreads / 32;
+    extern __shared__ __align__(1024) uint8_t ring[];
+    struct SlotInfo {
+        uint8_t *dst;
+        float *sdst;
+        int64_t ldy;
+        int32_t rows, cols;
+    };
+    __shared__ SlotInfo info[STAGES];
+    __shared__ __align__(8) uint64_t full[STAGES];
+    __shared__ __align__(8) uint64_t empty[STAGES];
+    __shared__ uint32_t red[2][2][NW];
+    __shared__ volatile int abort_flag;
+
+    const DescPack<MAXD> &p = P.p;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            dev::mbar_init(&full[s], 1);
+            dev::mbar_init(&empty[s], NW);
+        }
+        abort_flag = 0;
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        if (lane != 0) return;
+        int d = 0;
+        uint32_t k = 0;
+        bool dropped0 = false;
+        for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
+            const int st = (int)(k % STAGES);
+            const uint32_t round = k / STAGES;
+            if (round > 0 &&
+                !dev::mbar_wait_bounded(&empty[st], (round - 1) & 1u, p.wait_limit_ns, &abort_flag)) {
+                if (!abort_flag) {
+                    atomicOr(&g_error_word, 1u);
+                    abort_flag = 1;
+                }
+                break;
+            }
+            const Tile T = make_tile<ESIZE, 1, MAXD, 2>(p, w.t, d);
+            info[st].dst = T.dst;
+            info[st].sdst = T.sdst;
+            info[st].ldy = T.ldy;
+            info[st].rows = T.rows;
+            info[st].cols = T.cols;
+            dev::mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
+            if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
+                dropped0 = true;
+            else
+                dev::tma_load_3d(ring + (size_t)st * STAGE_BYTES, &P.maps[d], &full[st],
+                                 T.bj * BN, T.bi * BM, T.b);
+        }
+        const uint32_t issued = k;
+        for (int st = 0; st < STAGES && (uint32_t)st < issued; ++st) {
+            const uint32_t fills = (issued - (uint32_t)st + STAGES - 1) / STAGES;
+            if (dropped0 && st == 0 && fills == 1) continue;
+            if (!dev::mbar_wait_bounded(&full[st], (fills - 1) & 1u, kDrainLimitNs, nullptr))
+                atomicOr(&g_error_word, 2u);
+        }
+        return;
+    }
+
+    const int ct = threadIdx.x - 32;
+    const int cw = ct >> 5;
+    const int cv = ct & (VPR - 1);      // = lane
+    const int half = cv >> 4;           // block of this lane's columns
+    const int row0 = ct / VPR;          // = consumer warp index
+    const int colv = cv * VEC;          // column within the tile
+    const uint32_t hmask = half ? 0xffff0000u : 0x0000ffffu;
+    uint32_t k = 0;
+    for (TileWalk w(p.total_tiles); w.t < w.end; w.t += w.step, ++k) {
+        const int st = (int)(k % STAGES);
+        const bool ok = dev::mbar_wait_bounded(&full[st], (k / STAGES) & 1u, p.wait_limit_ns,
+                                               &abort_flag);
+        SlotInfo T = {nullptr, nullptr, 0, 0, 0};
+        if (ok) T = info[st];
+        uint4 R[V];
+        const uint8_t *stage = ring + (size_t)st * STAGE_BYTES;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int r = row0 + i * RSTEP;
+            R[i] = ok ? *reinterpret_cast<const uint4 *>(stage + ((size_t)r * COLS + colv) * ESIZE)
+                      : make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+        if (lane == 0 && ok) dev::mbar_arrive(&empty[st]);
+
+        uint32_t m = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE>(R));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(hmask, m, o));
+        if ((lane & 15) == 0) red[k & 1][half][cw] = m;
+        if (dev::named_bar_or(1, kTmaConsumerThreads, !ok)) {
+            if (ct == 0) {
+                atomicOr(&g_error_word, 1u);
+                abort_flag = 1;
+            }
+            break;
+        }
+        m = red[k & 1][half][0];
+#pragma unroll
+        for (int ww = 1; ww < NW; ++ww) m = max(m, red[k & 1][half][ww]);
+        if (half * BN >= T.cols) continue;  // second block beyond the matrix
+        float s, r;
+        dev::block_scale(m, kEps, s, r);
+        const uint64_t r2 = dev::splat2(r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int rr = row0 + i * RSTEP;
+            if (rr < T.rows && colv < T.cols)
+                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+        }
+        if ((ct & 15) == 0 && ct < 32) T.sdst[half] = s;
+    }
+}
+
 // ============================================================== launchers
 
 namespace {
@@ -727,10 +867,10 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
 }
 
 namespace {
-template <int ESIZE, int STAGES, int MODE>
-cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
+template <int ESIZE, int STAGES, int MODE, int MAXD>
+cudaError_t launch_tma_t(const TmaPack<MAXD> &p, cudaStream_t st) {
     constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
-    auto kern = k_tma<ESIZE, STAGES, MODE>;
+    auto kern = k_tma<ESIZE, STAGES, MODE, MAXD>;
     static cudaError_t attr =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
@@ -740,19 +880,39 @@ cudaError_t launch_tma_t(const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
 }
 }  // namespace
 
-cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<kMaxDescTma> &p, cudaStream_t st) {
+template <int MAXD>
+cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st) {
+    constexpr int S = FP8BQ_TMA_PAIR_STAGES;
+    constexpr size_t smem = (size_t)S * 128 * 256 * 2;
+    auto kern = k_tma_pair<S, MAXD>;
+    static cudaError_t attr =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
+    kern<<<grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <int MAXD>
+cudaError_t launch_tma(int esize, bool subwarp, const TmaPack<MAXD> &p, cudaStream_t st) {
     const int mode = subwarp ? MODE_SUB : p.p.group == 1 ? MODE_ONE : MODE_CTA;
     if (esize == 2) {
         constexpr int S = FP8BQ_TMA_STAGES_BF16;
-        return mode == MODE_ONE   ? launch_tma_t<2, S, MODE_ONE>(p, st)
-               : mode == MODE_SUB ? launch_tma_t<2, S, MODE_SUB>(p, st)
-                                  : launch_tma_t<2, S, MODE_CTA>(p, st);
+        return mode == MODE_ONE   ? launch_tma_t<2, S, MODE_ONE, MAXD>(p, st)
+               : mode == MODE_SUB ? launch_tma_t<2, S, MODE_SUB, MAXD>(p, st)
+                                  : launch_tma_t<2, S, MODE_CTA, MAXD>(p, st);
     }
     constexpr int S = FP8BQ_TMA_STAGES_F32;
-    return mode == MODE_ONE   ? launch_tma_t<4, S, MODE_ONE>(p, st)
-           : mode == MODE_SUB ? launch_tma_t<4, S, MODE_SUB>(p, st)
-                              : launch_tma_t<4, S, MODE_CTA>(p, st);
+    return mode == MODE_ONE   ? launch_tma_t<4, S, MODE_ONE, MAXD>(p, st)
+           : mode == MODE_SUB ? launch_tma_t<4, S, MODE_SUB, MAXD>(p, st)
+                              : launch_tma_t<4, S, MODE_CTA, MAXD>(p, st);
 }
+
+template cudaError_t launch_tma<kMaxDescSmall>(int, bool, const TmaPack<kMaxDescSmall> &,
+                                               cudaStream_t);
+template cudaError_t launch_tma<kMaxDescTma>(int, bool, const TmaPack<kMaxDescTma> &, cudaStream_t);
+template cudaError_t launch_tma_pair<kMaxDescSmall>(const TmaPack<kMaxDescSmall> &, cudaStream_t);
+template cudaError_t launch_tma_pair<kMaxDescTma>(const TmaPack<kMaxDescTma> &, cudaStream_t);
 
 cudaError_t read_and_clear_error_word(uint32_t *out) {
     uint32_t zero = 0;
