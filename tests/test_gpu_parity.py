@@ -223,3 +223,31 @@ def test_tma_bounded_wait_reports_timeout_and_recovers():
     (o2,) = run([sp], [ptr], fq.FP8BQ_PATH_TMA)
     assert_same(sp, o2.result(), want)
     del owner
+
+
+def test_grouped_call_replays_in_a_cuda_graph(qwen_layer_case):
+    """The grouped call only enqueues kernels (its descriptor table travels in
+    the kernel parameters), so once warmed up it can be captured in a CUDA
+    graph; replays write the same bytes as the oracle."""
+    from tests.gpu_util import Outputs
+    case = qwen_layer_case
+    outs = [Outputs(sp) for sp in case.specs]
+    descs = (fq.fp8bq_desc * len(outs))(*[o.desc(p) for o, p in zip(outs, case.ptrs)])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        assert fq.fp8bq_quantize_batched(descs, stream=s) == fq.FP8BQ_OK   # warm-up
+    s.synchronize()
+    for o in outs:                                   # clear the outputs before replaying
+        o.y.view.fill_(0)
+        o.s.view.fill_(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        st = fq.fp8bq_quantize_batched(descs, stream=s)
+    assert st == fq.FP8BQ_OK
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert fq.fp8bq_sync_status() == fq.FP8BQ_OK
+    for sp, o, w in zip(case.specs, outs, case.want):
+        assert_same(sp, o.result(), w)
