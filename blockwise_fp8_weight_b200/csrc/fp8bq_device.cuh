@@ -29,11 +29,6 @@ __device__ __forceinline__ void stg_stream_u32(void *p, uint32_t v) {
     asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// Bulk prefetch of `bytes` (multiple of 16, 16-byte aligned address) into L2.
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // ---------------------------------------------------------------- arithmetic
 //
 // The clamp of the method, clamp(x * r, -448, 448), is not issued as separate
@@ -157,38 +152,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// One probe that may suspend the thread in hardware for up to `hint_ns`
-// (it resumes as soon as the phase completes).
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity,
-                                                   uint32_t hint_ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok != 0;
-}
-
-#ifndef FP8BQ_WAIT_HINT_NS
-#define FP8BQ_WAIT_HINT_NS 0  // 0: the hardware's default suspend time
-#endif
-
 // Wait for a phase, giving up after `limit_ns` of global time or as soon as
 // *abort becomes nonzero.  Returns true if the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
                                                   uint64_t limit_ns,
                                                   const volatile int *abort) {
-    auto probe = [&]() {
-        return FP8BQ_WAIT_HINT_NS ? mbar_try_wait_hint(bar, parity, FP8BQ_WAIT_HINT_NS)
-                                  : mbar_try_wait(bar, parity);
-    };
-    if (probe()) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (probe()) return true;
+        if (mbar_try_wait(bar, parity)) return true;
         if (abort != nullptr && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
     }
@@ -202,10 +174,6 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
         " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(smem_dst)),
         "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
 // Named barrier over `count` threads.

@@ -35,9 +35,6 @@ constexpr uint64_t kDrainLimitNs = 2000000000ull;
 #ifndef FP8BQ_VEC_CTAS_PER_SM
 #define FP8BQ_VEC_CTAS_PER_SM 2   // resident 256-thread vector CTAs per SM
 #endif
-#ifndef FP8BQ_VEC_L2_PREFETCH
-#define FP8BQ_VEC_L2_PREFETCH 0   // vector kernel: bulk-prefetch the tile after next into L2
-#endif
 #ifndef FP8BQ_TMA_STAGES_BF16
 #define FP8BQ_TMA_STAGES_BF16 4   // 32 KB ring slots per TMA CTA (bf16 tiles)
 #endif
@@ -211,15 +208,6 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         }
     };
 
-    // Bulk-prefetch the rows of tile tn into L2 (a hint; no data dependence).
-    auto prefetch = [&](uint32_t tn) {
-        if (!FP8BQ_VEC_L2_PREFETCH || tn >= p.total_tiles) return;
-        int dd = d;
-        const Tile T = make_tile<ESIZE, G>(p, tn, dd);
-        for (int r = lane; r < T.rows; r += TEAM)
-            dev::prefetch_l2(T.src + (int64_t)r * T.ld * ESIZE, (uint32_t)(T.cols * ESIZE));
-    };
-
     auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
         const int bm = p.d[0].bm;
         uint32_t m[V];
@@ -282,7 +270,6 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         if (h1) {
             tb = make_tile<ESIZE, G>(p, t1, d);
             load(B, tb);
-            prefetch(t1 + stride);
         }
         process(A, ta, it++);
         if (!h1) break;
@@ -291,7 +278,6 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         if (h2) {
             ta = make_tile<ESIZE, G>(p, t2, d);
             load(A, ta);
-            prefetch(t2 + stride);
         }
         process(B, tb, it++);
         if (!h2) break;
@@ -388,24 +374,12 @@ __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ Des
     }
 }
 
-// The tiles one TMA CTA processes, in order: every gridDim.x-th tile
-// (strided), or one contiguous run of tiles per CTA.
-#ifndef FP8BQ_TMA_CONTIGUOUS
-#define FP8BQ_TMA_CONTIGUOUS 0
-#endif
+// The tiles one TMA CTA processes: every gridDim.x-th tile, starting at its
+// own index (a contiguous run of tiles per CTA measured no better).
 struct TileWalk {
     uint32_t t, end, step;
-    __device__ __forceinline__ explicit TileWalk(uint32_t total) {
-        if (FP8BQ_TMA_CONTIGUOUS) {
-            t = (uint32_t)((uint64_t)total * blockIdx.x / gridDim.x);
-            end = (uint32_t)((uint64_t)total * (blockIdx.x + 1) / gridDim.x);
-            step = 1;
-        } else {
-            t = blockIdx.x;
-            end = total;
-            step = gridDim.x;
-        }
-    }
+    __device__ __forceinline__ explicit TileWalk(uint32_t total)
+        : t(blockIdx.x), end(total), step(gridDim.x) {}
 };
 
 // ============================================================== TMA kernel
