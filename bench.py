@@ -109,6 +109,12 @@ def workload(name: str):
     if name == "qwen3_8b_layer":
         return W.qwen3_8b_layer(0, seed=1), ("one Qwen3-8B-shaped layer: 7 bf16 linear weights, "
                                              "block 128x128, one grouped launch")
+    if name == "qwen3_8b_layer_f32":
+        specs = W.qwen3_8b_layer(0, seed=1)
+        for sp in specs:
+            sp.dtype = "f32"
+        return specs, ("one Qwen3-8B-shaped layer in fp32 (7 linear weights), block 128x128, "
+                       "one grouped launch")
     if name == "moe_layer":
         return W.moe_layer(0), ("one Qwen3-30B-A3B-style MoE layer: q,k,v,o + 128-expert w13 "
                                 "and w2 stacks, bf16, block 128x128, one grouped launch")
@@ -455,12 +461,14 @@ def run_ours(args) -> None:
     dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
+        torch.cuda.nvtx.range_push(f"fp8bq timed steps x{args.steps}")
         t_start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
         t_end.record(stream)
+        torch.cuda.nvtx.range_pop()
         while not t_end.query():      # poll (not synchronize) so the sampler thread runs
             time.sleep(0.0005)
         torch.cuda.synchronize()
@@ -509,6 +517,7 @@ def run_ours(args) -> None:
         go.record(main)
         done = []
         for gi, g in enumerate(groups):
+            torch.cuda.nvtx.range_push(f"e2e layer {gi}")
             xl, xh = rng(lay.x_off, lambda i: specs[i].numel_storage * specs[i].elem_bytes, g)
             yl, yh = rng(lay.y_off, lambda i: specs[i].numel, g)
             sl, shh = rng(lay.s_off, lambda i: specs[i].nblocks * 4, g)
@@ -531,6 +540,7 @@ def run_ours(args) -> None:
                 e_o = torch.cuda.Event()
                 e_o.record(s_out)
             done.append(e_o)
+            torch.cuda.nvtx.range_pop()
         for e in done:
             main.wait_event(e)
 
@@ -571,7 +581,7 @@ def run_ours(args) -> None:
             "data": "synthetic",
             "config": {"workload": wl_desc, "name": args.workload, "tensors": len(specs),
                        "elements": elements, "bytes_per_step": bytes_per_step,
-                       "block": list(specs[0].block), "input_dtype": "bf16", "output_dtype": "e4m3fn",
+                       "block": list(specs[0].block), "input_dtype": specs[0].dtype, "output_dtype": "e4m3fn",
                        "path": args.path, "calls_per_step": args.mode,
                        "parallelism": f"replicas x{world}",
                        "l2": (f"no flush: {lay.x_bytes / 1e6:.0f} MB of inputs per step vs "
@@ -738,7 +748,8 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_model",
                     choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small",
-                             "act_1x128", "blk_64x64", "qkv", "ragged"])
+                             "act_1x128", "blk_64x64", "qkv", "ragged",
+                             "qwen3_8b_layer_f32"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",

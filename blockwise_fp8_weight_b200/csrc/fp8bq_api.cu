@@ -513,7 +513,8 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.gn = (int32_t)cdiv(D.N, D.block_n);
             o.begin = p.total;
             // vector: warp items of 32 x 16 codes per row; generic: one element
-            o.items = vector ? (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32)
+            o.items = vector ? (uint64_t)(D.batch * D.M) *
+                                   (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
                              : (uint64_t)(D.batch * D.M * D.N);
             p.total += o.items;
             ++p.n;

@@ -99,6 +99,8 @@ static_assert(sizeof(DequantPack<kMaxDescLarge>) < 32000, "kernel parameter limi
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st);
+// 16-byte code chunks per lane per warp work item of the vector dequant kernel
+int dequant_unroll();
 
 // Per-tensor scales (fp8bq_scale.cu): the tensors of a pack are cut into
 // work items of kScaleItem elements; every warp folds its items' absmax into
