@@ -146,6 +146,32 @@ __device__ __forceinline__ float group_scales(const uint32_t (&m)[V], int L, uin
     return sq;
 }
 
+// Reduce-scatter of 8 per-lane maxima over an aligned team of 16 lanes:
+// three halving exchange steps (xor 8, 4, 2) and one full step (xor 1).
+// Afterwards team lane q holds the team-wide max of slot 4*b3 + 2*b2 + b1
+// (b_k = bit k of q), i.e. slot q / 2; 8 shuffles instead of 32.
+__device__ __forceinline__ uint32_t reduce_scatter8x16(const uint32_t (&m)[8], uint32_t mask,
+                                                      int q) {
+    const bool h3 = q & 8, h2 = q & 4, h1 = q & 2;
+    uint32_t a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t send = h3 ? m[j] : m[j + 4];
+        const uint32_t keep = h3 ? m[j + 4] : m[j];
+        a[j] = max(keep, __shfl_xor_sync(mask, send, 8));
+    }
+    uint32_t b[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t send = h2 ? a[j] : a[j + 2];
+        const uint32_t keep = h2 ? a[j + 2] : a[j];
+        b[j] = max(keep, __shfl_xor_sync(mask, send, 4));
+    }
+    const uint32_t send = h1 ? b[0] : b[1];
+    uint32_t c = max(h1 ? b[1] : b[0], __shfl_xor_sync(mask, send, 2));
+    return max(c, __shfl_xor_sync(mask, c, 1));
+}
+
 // Quantize one 16-byte vector with rr = {r, r} and store its codes (8 bytes
 // for bf16, 4 for fp32).
 template <int ESIZE>
@@ -176,7 +202,7 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
-    static_assert(G == 1 || (G == V && TEAM <= 32), "per-slot blocks need a sub-warp team");
+    static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -209,17 +235,23 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     };
 
     auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
+      if constexpr (TEAM == 16 && V == 8) {  // the only stacked-block instantiation
         const int bm = p.d[0].bm;
         uint32_t m[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const uint4 one[1] = {R[i]};
             m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
-#pragma unroll
-            for (int o = TEAM / 2; o > 0; o >>= 1) m[i] = max(m[i], __shfl_xor_sync(shfl_mask, m[i], o));
         }
+        // lane q ends with the max of slot q / 2, computes its scale, and the
+        // reciprocal of slot i is fetched from lane 2 i of the team
+        const uint32_t mq = reduce_scatter8x16(m, shfl_mask, lane);
+        float s_mine, r_mine;
+        dev::block_scale(mq, kEps, s_mine, r_mine);
+        const int base = (threadIdx.x & 31) & ~(TEAM - 1);
         float r[V];
-        const float s_mine = group_scales<V>(m, TEAM, shfl_mask, r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + 2 * i);
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             if (i * bm >= T.rows) break;  // blocks below the matrix
@@ -227,7 +259,9 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             if (rr < T.rows && colv < T.cols)
                 vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv);
         }
-        if (lane < V && lane * bm < T.rows) T.sdst[(int64_t)lane * p.d[0].gn] = s_mine;
+        const int slot = lane >> 1;
+        if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * p.d[0].gn] = s_mine;
+      }
     };
 
     auto process = [&](const uint4 (&R)[V], const Tile &T, uint32_t it) {
