@@ -50,10 +50,16 @@ fp8bq_status check_desc(const fp8bq_desc &D, bool *empty) {
     if (D.x == nullptr || D.y_u8 == nullptr || D.descale_f32 == nullptr) return FP8BQ_ERR_NULL;
     const int es = esize_of(D.dtype_in);
     if (((uintptr_t)D.x % es) != 0 || ((uintptr_t)D.descale_f32 % 4) != 0) return FP8BQ_ERR_ALIGN;
-    if (D.batch > 1) {
-        const int64_t gm = cdiv(D.M, D.block_m), gn = cdiv(D.N, D.block_n);
-        if (D.y_batch_stride < D.M * D.N || D.s_batch_stride < gm * gn) return FP8BQ_ERR_OVERLAP;
-    }
+    // every byte offset the kernels form must fit comfortably in 64 bits
+    const int64_t gm = cdiv(D.M, D.block_m), gn = cdiv(D.N, D.block_n);
+    const __int128 b1 = D.batch - 1, lim = (__int128)1 << 62;
+    const bool multi = D.batch > 1;
+    if ((b1 * (multi ? D.x_batch_stride : 0) + (__int128)(D.M - 1) * D.ld + D.N) * es > lim ||
+        b1 * (multi ? D.y_batch_stride : 0) + (__int128)D.M * D.N > lim ||
+        (b1 * (multi ? D.s_batch_stride : 0) + (__int128)gm * gn) * 4 > lim)
+        return FP8BQ_ERR_SHAPE;
+    if (multi && (D.y_batch_stride < D.M * D.N || D.s_batch_stride < gm * gn))
+        return FP8BQ_ERR_OVERLAP;
     return FP8BQ_OK;
 }
 
@@ -478,6 +484,11 @@ fp8bq_status check_dequant_desc(const fp8bq_dequant_desc &D, bool *empty) {
     if (D.y_u8 == nullptr || D.descale_f32 == nullptr || D.out == nullptr) return FP8BQ_ERR_NULL;
     if ((uintptr_t)D.descale_f32 % 4 || (uintptr_t)D.out % esize_of(D.dtype_out))
         return FP8BQ_ERR_ALIGN;
+    const __int128 b1 = D.batch - 1, lim = (__int128)1 << 62;
+    if ((b1 * (D.batch > 1 ? D.out_batch_stride : 0) + (__int128)(D.M - 1) * D.ld_out + D.N) *
+                esize_of(D.dtype_out) > lim ||
+        (__int128)D.batch * D.M * D.N > lim)
+        return FP8BQ_ERR_SHAPE;
     return FP8BQ_OK;
 }
 
@@ -627,7 +638,7 @@ fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out
     for (int i = 0; i < n; ++i) {
         const fp8bq_scale_desc &D = t[i];
         if (D.dtype_in != FP8BQ_BF16 && D.dtype_in != FP8BQ_F32) return FP8BQ_ERR_DTYPE;
-        if (D.numel < 0) return FP8BQ_ERR_SHAPE;
+        if (D.numel < 0 || D.numel > ((int64_t)1 << 60)) return FP8BQ_ERR_SHAPE;
         if (D.numel == 0) continue;
         if (D.x == nullptr) return FP8BQ_ERR_NULL;
         const int es = esize_of(D.dtype_in);

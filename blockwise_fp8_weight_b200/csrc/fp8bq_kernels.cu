@@ -54,6 +54,7 @@ struct Tile {
     int64_t ldy;      // output row stride (= N)
     int rows, cols;   // valid extent
     int b, bi, bj;    // coordinates (TMA)
+    int gn;           // descale row length (blocks per matrix row)
 };
 
 // Tile t of a launch.  A tile is G vertically adjacent blocks of one matrix
@@ -88,6 +89,7 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     T.b = (int)b;
     T.bi = (int)bi;
     T.bj = (int)bj;
+    T.gn = D.gn;
     return T;
 }
 
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
                 vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv);
         }
         const int slot = lane >> 1;
-        if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * p.d[0].gn] = s_mine;
+        if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
       }
     };
 

@@ -33,9 +33,13 @@
  * device memory per call, and keeps no pointer after a call returns.
  *
  * Execution: calls are asynchronous on `stream`, like a kernel launch.  All
- * arguments are checked before anything is launched; a call that returns an
- * error launched nothing.  Inputs must not overlap outputs, and outputs must
- * not overlap each other (checked on the address ranges each argument spans).
+ * arguments are checked before anything is launched: a call that returns an
+ * argument error (anything but FP8BQ_ERR_DEVICE) launched nothing.  A call may
+ * enqueue several launches (one per kernel variant in a grouped call); if the
+ * CUDA runtime rejects one of them the call returns FP8BQ_ERR_DEVICE and the
+ * launches before it stay enqueued.  Inputs must not overlap outputs, and
+ * outputs must not overlap each other (checked on the address ranges each
+ * argument spans).
  * NaN and infinite inputs are outside the contract (no error, unspecified
  * codes).
  */
@@ -66,7 +70,8 @@ typedef enum fp8bq_status {
     FP8BQ_OK = 0,
     FP8BQ_ERR_NULL = 1,           /* a required pointer is NULL */
     FP8BQ_ERR_SHAPE = 2,          /* M, N, batch or a stride negative; ld < N; M or N >= 2^31;
-                                     too many blocks in one tensor (>= 2^31) */
+                                     too many blocks in one tensor (>= 2^31); an argument's
+                                     byte extent beyond 2^62 */
     FP8BQ_ERR_BLOCK = 3,          /* block_m or block_n < 1, or block_m * block_n > 65536 */
     FP8BQ_ERR_DTYPE = 4,          /* dtype_in not an fp8bq_dtype */
     FP8BQ_ERR_OVERLAP = 5,        /* an output overlaps an input or another output */
@@ -132,8 +137,8 @@ typedef struct fp8bq_desc {
  *   desc_table   HOST memory, n_tensors entries; read during the call only.
  *   n_tensors    >= 0.
  *
- * Either every tensor is checked and the whole list is enqueued, or an error
- * is returned and nothing is launched.
+ * Every tensor is checked before the first launch; an argument error in any
+ * descriptor rejects the whole list and nothing is launched.
  */
 FP8BQ_API fp8bq_status fp8bq_quantize_batched(const fp8bq_desc *desc_table, int n_tensors,
                                     cudaStream_t stream);

@@ -71,6 +71,7 @@ def q(**kw):
     (dict(N=-1, ld=0), fq.FP8BQ_ERR_SHAPE),
     (dict(ld=383), fq.FP8BQ_ERR_SHAPE),
     (dict(M=1 << 31, N=1, ld=1), fq.FP8BQ_ERR_SHAPE),
+    (dict(M=1 << 30, N=4, ld=1 << 40), fq.FP8BQ_ERR_SHAPE),   # byte offsets beyond 2^62
     (dict(x=0), fq.FP8BQ_ERR_NULL),
     (dict(y_u8=0), fq.FP8BQ_ERR_NULL),
     (dict(descale_f32=0), fq.FP8BQ_ERR_NULL),

@@ -251,3 +251,31 @@ def test_grouped_call_replays_in_a_cuda_graph(qwen_layer_case):
     assert fq.fp8bq_sync_status() == fq.FP8BQ_OK
     for sp, o, w in zip(case.specs, outs, case.want):
         assert_same(sp, o.result(), w)
+
+
+@pytest.mark.parametrize("block", [(128, 128), (1, 128), (64, 64)])
+@pytest.mark.parametrize("path", ["auto", "vector", "generic"])
+def test_many_tensors_in_one_call(path, block):
+    """700 tensors of mixed shapes in one grouped call: the list is split into
+    several launches (320 descriptors per vector/generic pack, 128 per TMA
+    pack), tensors of different widths share a launch, and every tensor still
+    matches the oracle."""
+    rng = np.random.default_rng(101)
+    specs = []
+    for i in range(700):
+        M = int(rng.integers(1, 5)) * 128 + int(rng.integers(0, 2)) * int(rng.integers(1, 127))
+        N = int(rng.choice([128, 256, 384, 1024]))
+        specs.append(TensorSpec(f"many.{i}", M, N, block=block, seed=111, tensor_id=i,
+                                sigma=0.02, outlier_p=1e-3))
+    hosts = [W.materialize(sp) for sp in specs]
+    # one device buffer for all inputs, 256-byte aligned offsets
+    offs, o = [], 0
+    for x in hosts:
+        offs.append(o)
+        o += (x.nbytes + 255) // 256 * 256
+    buf = torch.empty(o, dtype=torch.uint8, device="cuda")
+    for x, off in zip(hosts, offs):
+        buf[off:off + x.nbytes].copy_(torch.from_numpy(x.view(np.uint8)))
+    outs = run(specs, [buf.data_ptr() + off for off in offs], PATHS[path])
+    for sp, x, out in zip(specs, hosts, outs):
+        assert_same(sp, out.result(), oracle_expected(sp, x))
