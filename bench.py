@@ -410,6 +410,12 @@ def run_ours(args) -> None:
     dev = torch.device("cuda", local_rank)
     dist = Dist(world, "nccl", dev)
     specs, wl_desc = workload(args.workload)
+    if args.repeat > 1:  # the same tensor list args.repeat times, fresh values each time
+        import dataclasses
+        specs = [dataclasses.replace(sp, name=f"{sp.name}.r{k}", tensor_id=sp.tensor_id + 4096 * k,
+                                     meta=dict(sp.meta, layer=k))
+                 for k in range(args.repeat) for sp in specs]
+        wl_desc += f", x{args.repeat} in one call"
     lay = Layout(specs)
     bytes_per_step = sum(sp.algorithmic_bytes for sp in specs)
     elements = sum(sp.numel for sp in specs)
@@ -752,6 +758,8 @@ def main() -> None:
                              "qwen3_8b_layer_f32"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--repeat", type=int, default=1,
+                    help="replicate the workload's tensor list this many times (distinct values)")
     ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",
                     help="C-ABI calls per step: one grouped call, one per layer, or one per "
                          "tensor")
