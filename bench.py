@@ -126,6 +126,10 @@ def workload(name: str):
     if name == "ragged":
         sp = [t for t in W.edge() if t.name == "edge.bf16.4000x4100"]
         return sp, "bf16 4000x4100 (rows only 8-byte aligned), block 128x128, Student-t(3) x 0.02"
+    if name == "edge":
+        return W.edge(), ("ragged and small-block edge set in one grouped call: bf16 and fp32 "
+                          "4000x4100, 130x129, 1x128, 12345x4096, 4000x4100 with ld 4164 "
+                          "(block 128x128), bf16 16384x4096 with [1,128] and [64,64] blocks")
     if name in ("act_1x128", "blk_64x64"):
         sp = [t for t in W.edge() if t.name.endswith("b1x128" if name == "act_1x128" else "b64x64")]
         return sp, f"bf16 16384x4096, N(0,1) x row lognormal(0,1), blocks {sp[0].block}"
@@ -362,13 +366,26 @@ def build_descs(specs, lay: Layout, x_base: int, y_base: int, s_base: int, idx=N
 
 
 def count_launches(arr) -> int:
+    """Kernel launches of one fp8bq_quantize_batched call over `arr`, grouped the
+    way the library groups tensors: by kernel path and input dtype; then by
+    block shape and, for the vector kernel, by 16-byte or 8-byte-halves row
+    alignment; generic blocks by size class (one CTA per block from 2048
+    elements).  A group launches once per pack of 128 (TMA) or 320 tensors."""
     import blockwise_fp8_weight_b200 as fq
     groups: dict = {}
     for d in arr:
         p = fq.fp8bq_path_for(d)
-        key = (p, d.dtype_in, d.block_m if p != 3 else 0, d.block_n if p != 3 else 0)
+        if p == fq.FP8BQ_PATH_GENERIC:
+            key = (p, d.dtype_in, d.block_m * d.block_n >= 2048)
+        else:
+            es = 2 if d.dtype_in == fq.FP8BQ_BF16 else 4
+            vec = 16 // es
+            a16 = (d.x % 16 == 0 and d.ld * es % 16 == 0 and d.N % vec == 0 and d.y_u8 % vec == 0
+                   and (d.batch == 1 or (d.x_batch_stride * es % 16 == 0
+                                         and d.y_batch_stride % vec == 0)))
+            key = (p, d.dtype_in, d.block_m, d.block_n, p == fq.FP8BQ_PATH_VECTOR and not a16)
         groups[key] = groups.get(key, 0) + 1
-    return sum(-(-n // (128 if k[0] == 2 else 320)) for k, n in groups.items())
+    return sum(-(-n // (128 if k[0] == fq.FP8BQ_PATH_TMA else 320)) for k, n in groups.items())
 
 
 def cpu_baseline(specs, host: np.ndarray, lay: Layout, seconds: float) -> dict:
@@ -754,7 +771,7 @@ def main() -> None:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_model",
                     choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small",
-                             "act_1x128", "blk_64x64", "qkv", "ragged",
+                             "act_1x128", "blk_64x64", "qkv", "ragged", "edge",
                              "qwen3_8b_layer_f32"])
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)

@@ -145,6 +145,18 @@ bool vector_aligned(const fp8bq_desc &D) {
     return true;
 }
 
+// The weaker alignment of the vector kernel's HALVES mode: 8-byte input rows
+// and output pieces of half a vector (4 codes for bf16, 2 for fp32), so every
+// row holds a whole number of 8-byte input halves (bf16 rows of 4100
+// elements, say).
+bool halves_aligned(const fp8bq_desc &D) {
+    const int es = esize_of(D.dtype_in), half = 8 / es;
+    if ((uintptr_t)D.x % 8 || (D.ld * es) % 8 || D.N % half) return false;
+    if ((uintptr_t)D.y_u8 % half) return false;
+    if (D.batch > 1 && ((D.x_batch_stride * es) % 8 || D.y_batch_stride % half)) return false;
+    return true;
+}
+
 Variant vector_variant(const fp8bq_desc &D) {
     for (Variant v : {Variant::VecT16, Variant::VecT64, Variant::VecTBig})
         if (vector_fits(D, v)) return v;
@@ -199,7 +211,7 @@ Variant choose(const fp8bq_desc &D, int path) {
     if (path == FP8BQ_PATH_AUTO && tma && g == 1 &&
         (int64_t)D.block_m * D.block_n * esize_of(D.dtype_in) >= kTmaMinSlotBytes)
         return Variant::Tma;
-    if (!vector_aligned(D)) return Variant::Generic;
+    if (!vector_aligned(D) && !halves_aligned(D)) return Variant::Generic;
     return vector_variant(D);
 }
 
@@ -351,8 +363,8 @@ void pack_header(DescPack<MAXD> &p) {
 // Launch one group (same variant, dtype and, for vector/TMA, block shape) in
 // chunks that fit the parameter pack and keep the tile count below 2^31.
 template <int MAXD>
-cudaError_t launch_group(Variant v, int es, const fp8bq_desc *t, const std::vector<int> &idx,
-                         cudaStream_t st) {
+cudaError_t launch_group(Variant v, int es, bool halves, const fp8bq_desc *t,
+                         const std::vector<int> &idx, cudaStream_t st) {
     static thread_local DescPack<MAXD> p;  // large: keep it off the stack
     size_t i = 0;
     while (i < idx.size()) {
@@ -367,7 +379,7 @@ cudaError_t launch_group(Variant v, int es, const fp8bq_desc *t, const std::vect
             ++i;
         }
         const cudaError_t e = v == Variant::Generic ? launch_generic<MAXD>(es, p, st)
-                                                    : launch_vector<MAXD>(v, es, p, st);
+                                                    : launch_vector<MAXD>(v, es, halves, p, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -404,8 +416,9 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
 struct GroupKey {
     Variant v;
     int es, bm, bn;
+    bool halves;
     bool operator==(const GroupKey &o) const {
-        return v == o.v && es == o.es && bm == o.bm && bn == o.bn;
+        return v == o.v && es == o.es && bm == o.bm && bn == o.bn && halves == o.halves;
     }
 };
 
@@ -441,8 +454,9 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         // vector / TMA launches need one block shape; generic ones only one
         // size class (CTA per block for >= 2048 elements, else warp per block)
         const bool big = (int64_t)D.block_m * D.block_n >= 2048;
+        const bool halves = v != Variant::Generic && v != Variant::Tma && !vector_aligned(D);
         GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? (int)big : D.block_m,
-                   v == Variant::Generic ? 0 : D.block_n};
+                   v == Variant::Generic ? 0 : D.block_n, halves};
         size_t g = 0;
         while (g < keys.size() && !(keys[g] == k)) ++g;
         if (g == keys.size()) {
@@ -460,9 +474,11 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
                     ? launch_tma_group<kMaxDescSmall>(keys[g].es, table, members[g], maps[g], stream)
                     : launch_tma_group<kMaxDescTma>(keys[g].es, table, members[g], maps[g], stream);
         else if (members[g].size() <= (size_t)kMaxDescSmall)
-            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, table, members[g], stream);
+            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].halves, table,
+                                            members[g], stream);
         else
-            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, table, members[g], stream);
+            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].halves, table,
+                                            members[g], stream);
         if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
     }
     return FP8BQ_OK;

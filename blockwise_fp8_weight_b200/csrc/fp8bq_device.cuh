@@ -21,12 +21,24 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
     return v;
 }
 
+// 8-byte load on the read-only path for rows that are only 8-byte aligned.
+// It allocates in L1: the two 8-byte halves of a lane's 16 bytes are read by
+// two loads, and the second one finds the sectors of the first in L1.
+__device__ __forceinline__ uint2 ldg_v2(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
 // Streaming (evict-first) stores of the e4m3fn codes.
 __device__ __forceinline__ void stg_stream_v2(void *p, uint2 v) {
     asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 __device__ __forceinline__ void stg_stream_u32(void *p, uint32_t v) {
     asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void stg_stream_u16(void *p, uint16_t v) {
+    asm volatile("st.global.cs.u16 [%0], %1;" ::"l"(p), "h"(v) : "memory");
 }
 
 // ---------------------------------------------------------------- arithmetic

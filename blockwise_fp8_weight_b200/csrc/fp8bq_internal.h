@@ -64,8 +64,10 @@ enum class Variant : int {
 };
 
 // Launchers (fp8bq_kernels.cu).  Each returns cudaSuccess or the launch error.
+// halves: rows only 8-byte aligned (each 16-byte vector moved as two halves)
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st);
+cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
+                          cudaStream_t st);
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
 template <int MAXD>

@@ -188,6 +188,22 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
     }
 }
 
+// The same for a lane's 16 bytes held as two 8-byte halves (rows that are
+// only 8-byte aligned): each half is quantized and stored on its own, the
+// upper one only when hi_ok (it lies inside the row).  Codes: 4 bytes per
+// bf16 half, 2 per fp32 half.
+template <int ESIZE>
+__device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t rr, uint8_t *dst,
+                                                       bool hi_ok) {
+    if constexpr (ESIZE == 2) {
+        dev::stg_stream_u32(dst, dev::quant_bf16x4(v.x, v.y, rr));
+        if (hi_ok) dev::stg_stream_u32(dst + 4, dev::quant_bf16x4(v.z, v.w, rr));
+    } else {
+        dev::stg_stream_u16(dst, dev::quant_pair_bits(v.x, v.y, rr));
+        if (hi_ok) dev::stg_stream_u16(dst + 2, dev::quant_pair_bits(v.z, v.w, rr));
+    }
+}
+
 // ============================================================== vector kernel
 //
 // A team of TEAM threads owns one block at a time; a block of bm x bn
@@ -201,7 +217,11 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
 // G > 1 (small blocks): a tile is G vertically adjacent blocks and slot i of
 // every thread holds a vector of block i (one block is exactly one row-step
 // of the team, bm * vpr == TEAM), so each slot is reduced on its own.
-template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
+//
+// HALVES (rows only 8-byte aligned; N a multiple of VEC / 2): the same
+// geometry, each 16-byte vector moved as two 8-byte halves; a half beyond
+// the row end reads as zeros (no effect on the absmax) and is not stored.
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
@@ -225,14 +245,31 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         TEAM >= 32 ? 0xffffffffu : (((1u << TEAM) - 1u) << ((threadIdx.x & 31) & ~(TEAM - 1)));
     int d = 0;  // current descriptor; advances monotonically with the tile id
 
+    // upper 8-byte half of this lane's vector inside the row (HALVES only)
+    auto hi_ok = [&](const Tile &T) { return colv + VEC / 2 < T.cols; };
+    auto store = [&](const uint4 &v, uint64_t rr, uint8_t *dst, const Tile &T) {
+        if constexpr (HALVES)
+            vec_quant_store_halves<ESIZE>(v, rr, dst, hi_ok(T));
+        else
+            vec_quant_store<ESIZE>(v, rr, dst);
+    };
+
     auto load = [&](uint4 (&R)[V], const Tile &T) {
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int r = row0 + i * rstep;
-            if (r < T.rows && colv < T.cols)
-                R[i] = dev::ldg_stream_v4(T.src + ((int64_t)r * T.ld + colv) * ESIZE);
-            else
+            if (r < T.rows && colv < T.cols) {
+                const char *a = T.src + ((int64_t)r * T.ld + colv) * ESIZE;
+                if constexpr (HALVES) {
+                    const uint2 lo = dev::ldg_v2(a);
+                    const uint2 hi = hi_ok(T) ? dev::ldg_v2(a + 8) : make_uint2(0u, 0u);
+                    R[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+                } else {
+                    R[i] = dev::ldg_stream_v4(a);
+                }
+            } else {
                 R[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
     };
 
@@ -259,7 +296,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             if (i * bm >= T.rows) break;  // blocks below the matrix
             const int rr = row0 + i * rstep;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv);
+                store(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv, T);
         }
         const int slot = lane >> 1;
         if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
@@ -290,7 +327,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         for (int i = 0; i < V; ++i) {
             const int rr = row0 + i * rstep;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+                store(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv, T);
         }
         if (lane == 0) *T.sdst = s;
     };
@@ -822,31 +859,38 @@ unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {
     return (unsigned)(need < cap ? (need ? need : 1) : cap);
 }
 
-template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
-cudaError_t launch_vector_t(const DescPack<MAXD> &p, cudaStream_t st) {
-    auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD>;
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
+cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
+    auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES>;
     static int occ = resident_ctas(kern, CTA, 0);
     const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
     kern<<<grid, CTA, 0, st>>>(p);
     return cudaGetLastError();
 }
 
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
+cudaError_t launch_vector_t(bool halves, const DescPack<MAXD> &p, cudaStream_t st) {
+    return halves ? launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true>(p, st)
+                  : launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, false>(p, st);
+}
+
 }  // namespace
 
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, const DescPack<MAXD> &p, cudaStream_t st) {
+cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
+                          cudaStream_t st) {
     if (esize == 2) {
         switch (v) {
-            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(p, st);
-            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(p, st);
-            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(p, st);
+            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(halves, p, st);
+            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(halves, p, st);
+            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(halves, p, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (v) {
-        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(p, st);
-        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(p, st);
-        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(p, st);
+        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(halves, p, st);
+        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(halves, p, st);
+        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(halves, p, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -932,9 +976,11 @@ cudaError_t read_and_clear_error_word(uint32_t *out) {
     return e;
 }
 
-template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, const DescPack<kMaxDescSmall> &,
+template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, bool,
+                                                  const DescPack<kMaxDescSmall> &,
                                                   cudaStream_t);
-template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, const DescPack<kMaxDescLarge> &,
+template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, bool,
+                                                  const DescPack<kMaxDescLarge> &,
                                                   cudaStream_t);
 template cudaError_t launch_generic<kMaxDescSmall>(int, const DescPack<kMaxDescSmall> &,
                                                    cudaStream_t);

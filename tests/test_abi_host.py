@@ -154,10 +154,21 @@ def test_variant_choice(path_guard):
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_VECTOR) == fq.FP8BQ_OK
     assert P(desc()) == fq.FP8BQ_PATH_VECTOR
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO) == fq.FP8BQ_OK
-    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC   # rows only 8-B aligned
-    assert P(desc(batch=1, N=4096, ld=4100)) == fq.FP8BQ_PATH_GENERIC
+    # rows only 8-byte aligned: the vector kernel in 8-byte halves
+    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(batch=1, N=4096, ld=4100)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(x=X + 8)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(y_u8=Y + 4)) == fq.FP8BQ_PATH_VECTOR
+    assert P(desc(batch=1, N=4100, ld=4100, dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
+    assert P(desc(batch=1, N=4098, ld=4098, dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_VECTOR
+    # narrower than that: the generic kernel
+    assert P(desc(batch=1, N=4102, ld=4102)) == fq.FP8BQ_PATH_GENERIC   # rows 4-byte aligned
+    assert P(desc(batch=1, N=4097, ld=4100)) == fq.FP8BQ_PATH_GENERIC   # codes rows odd
+    assert P(desc(batch=1, N=4097, ld=4097, dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_GENERIC
     assert P(desc(x=X + 2)) == fq.FP8BQ_PATH_GENERIC
-    assert P(desc(y_u8=Y + 4)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(x=X + 4)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(y_u8=Y + 2)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(x_batch_stride=1536 * 2048 + 2)) == fq.FP8BQ_PATH_GENERIC
     assert P(desc(batch=1, block_m=5, block_n=7)) == fq.FP8BQ_PATH_GENERIC
     assert P(desc(batch=1, block_m=256, block_n=256)) == fq.FP8BQ_PATH_GENERIC  # 65536 elements
     assert P(desc(block_m=0)) == -1
@@ -166,7 +177,8 @@ def test_variant_choice(path_guard):
     assert P(desc(dtype_in=fq.FP8BQ_F32)) == fq.FP8BQ_PATH_TMA
     assert P(desc(batch=1, block_m=1, block_n=128)) == fq.FP8BQ_PATH_TMA    # stacked blocks
     assert P(desc(batch=1, block_m=64, block_n=64)) == fq.FP8BQ_PATH_TMA
-    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_GENERIC
+    assert P(desc(batch=1, N=4100, ld=4100)) == fq.FP8BQ_PATH_VECTOR   # no tensor map
+    assert P(desc(batch=1, N=4102, ld=4102)) == fq.FP8BQ_PATH_GENERIC
     assert fq.fp8bq_set_path(fq.FP8BQ_PATH_GENERIC) == fq.FP8BQ_OK
     assert P(desc()) == fq.FP8BQ_PATH_GENERIC
     assert fq.fp8bq_set_path(7) == fq.FP8BQ_ERR_ARG

@@ -15,7 +15,7 @@ import blockwise_fp8_weight_b200 as fq
 import oracle
 from synth import TensorSpec, DIST_STUDENT_T3
 from synth import workloads as W
-from tests.gpu_util import assert_same, oracle_expected, run, to_device
+from tests.gpu_util import Outputs, assert_same, oracle_expected, run, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -109,6 +109,32 @@ def test_misaligned_pointers(dtype, xoff, yoff):
     want = oracle_expected(sp, x)
     for path in PATHS.values():
         (o,) = run([sp], [ptr], path, y_offsets=[yoff])
+        assert_same(sp, o.result(), want)
+    del owner
+
+
+@pytest.mark.parametrize("dtype,M,N,ld,block,batch", [
+    ("bf16", 300, 4100, None, (128, 128), 1),   # last vector of a row: upper half outside
+    ("bf16", 200, 1028, 1036, (64, 64), 1),     # padded rows (poison in the padding)
+    ("bf16", 37, 516, None, (1, 128), 1),       # stacked 1x128 blocks, ragged stack
+    ("bf16", 130, 4100, None, (128, 128), 3),   # expert stack, 8-byte-aligned strides
+    ("f32", 300, 4098, None, (128, 128), 1),
+    ("f32", 200, 1030, 1034, (64, 64), 1),
+    ("f32", 37, 514, None, (1, 128), 1),
+])
+def test_half_vector_rows(dtype, M, N, ld, block, batch):
+    """Rows that are 8-byte but not 16-byte aligned take the vector kernel in
+    8-byte halves; where a row ends inside a vector its upper half is neither
+    read nor written."""
+    sp = TensorSpec(f"half.{dtype}.{batch}x{M}x{N}.b{block[0]}x{block[1]}", M, N, batch=batch,
+                    ld=ld, dtype=dtype, block=block, seed=73, tensor_id=M * 131 + N,
+                    dist=DIST_STUDENT_T3)
+    x = W.materialize(sp)
+    owner, ptr = to_device(x)
+    assert fq.fp8bq_path_for(Outputs(sp).desc(ptr)) == fq.FP8BQ_PATH_VECTOR
+    want = oracle_expected(sp, x)
+    for path in (PATHS["auto"], PATHS["vector"]):
+        (o,) = run([sp], [ptr], path)
         assert_same(sp, o.result(), want)
     del owner
 
