@@ -131,6 +131,10 @@ def lib() -> ctypes.CDLL:
             L.fp8bq_set_path.restype = i32
             L.fp8bq_get_path.argtypes = []
             L.fp8bq_get_path.restype = i32
+            L.fp8bq_set_pdl.argtypes = [i32]
+            L.fp8bq_set_pdl.restype = i32
+            L.fp8bq_get_pdl.argtypes = []
+            L.fp8bq_get_pdl.restype = i32
             L.fp8bq_path_for.argtypes = [ctypes.POINTER(fp8bq_desc)]
             L.fp8bq_path_for.restype = i32
             L.fp8bq_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
@@ -223,6 +227,14 @@ def fp8bq_set_path(path: int) -> int:
 
 def fp8bq_get_path() -> int:
     return lib().fp8bq_get_path()
+
+
+def fp8bq_set_pdl(enable: int) -> int:
+    return lib().fp8bq_set_pdl(int(enable))
+
+
+def fp8bq_get_pdl() -> int:
+    return lib().fp8bq_get_pdl()
 
 
 def fp8bq_path_for(desc: fp8bq_desc) -> int:

@@ -26,6 +26,7 @@ namespace {
 std::atomic<int> g_path{FP8BQ_PATH_AUTO};
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<uint32_t> g_inject{0};
+std::atomic<int> g_pdl{1};
 
 int esize_of(int32_t dtype) { return dtype == FP8BQ_BF16 ? 2 : 4; }
 
@@ -686,6 +687,8 @@ fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out
 
 }  // namespace
 
+bool fp8bq::pdl_enabled() { return g_pdl.load(std::memory_order_relaxed) != 0; }
+
 extern "C" {
 
 fp8bq_status fp8bq_tensor_scale(const fp8bq_scale_desc *desc_table, int n_tensors,
@@ -781,6 +784,13 @@ fp8bq_status fp8bq_set_path(fp8bq_path path) {
 }
 
 fp8bq_path fp8bq_get_path(void) { return (fp8bq_path)g_path.load(); }
+
+fp8bq_status fp8bq_set_pdl(int enable) {
+    g_pdl.store(enable ? 1 : 0);
+    return FP8BQ_OK;
+}
+
+int fp8bq_get_pdl(void) { return g_pdl.load(); }
 
 int fp8bq_path_for(const fp8bq_desc *desc) {
     if (desc == nullptr) return -1;

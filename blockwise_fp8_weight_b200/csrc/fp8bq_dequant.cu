@@ -8,6 +8,7 @@
 //
 // decode() is exact in two steps: cvt.rn.f16x2.e4m3x2 (every e4m3fn value,
 // subnormals included, is a normal fp16 value) and fp16 -> fp32.
+#include "fp8bq_device.cuh"
 #include "fp8bq_internal.h"
 
 namespace fp8bq {
@@ -60,6 +61,7 @@ constexpr int kDqUnroll = FP8BQ_DQ_UNROLL;
 
 template <int OES, int MAXD>
 __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ DequantPack<MAXD> p) {
+    dev::pdl_entry();
     constexpr int U = kDqUnroll;
     const int lane = threadIdx.x & 31;
     const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
@@ -129,6 +131,7 @@ __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ Deq
 template <int OES, int MAXD>
 __global__ void __launch_bounds__(256)
     k_dequant_generic(const __grid_constant__ DequantPack<MAXD> p) {
+    dev::pdl_entry();
     int d = 0;
     for (uint64_t k = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; k < p.total;
          k += (uint64_t)gridDim.x * blockDim.x) {
@@ -171,18 +174,11 @@ int dequant_unroll() { return kDqUnroll; }
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st) {
     const unsigned grid = dq_grid(vector ? p.total * 32 : p.total);  // vector: a warp per item
-    if (vector) {
-        if (out_esize == 2)
-            k_dequant_vec<2, MAXD><<<grid, 256, 0, st>>>(p);
-        else
-            k_dequant_vec<4, MAXD><<<grid, 256, 0, st>>>(p);
-    } else {
-        if (out_esize == 2)
-            k_dequant_generic<2, MAXD><<<grid, 256, 0, st>>>(p);
-        else
-            k_dequant_generic<4, MAXD><<<grid, 256, 0, st>>>(p);
-    }
-    return cudaGetLastError();
+    if (vector)
+        return out_esize == 2 ? launch_kernel(k_dequant_vec<2, MAXD>, grid, 256, 0, st, p)
+                              : launch_kernel(k_dequant_vec<4, MAXD>, grid, 256, 0, st, p);
+    return out_esize == 2 ? launch_kernel(k_dequant_generic<2, MAXD>, grid, 256, 0, st, p)
+                          : launch_kernel(k_dequant_generic<4, MAXD>, grid, 256, 0, st, p);
 }
 
 template cudaError_t launch_dequant<kMaxDescSmall>(const DequantPack<kMaxDescSmall> &, int, bool,

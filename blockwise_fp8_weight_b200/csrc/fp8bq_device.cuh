@@ -9,6 +9,17 @@
 namespace fp8bq {
 namespace dev {
 
+// ---------------------------------------------------------------- launch order
+
+// First statement of every kernel: allow the next kernel of the stream to
+// launch (its own wait keeps it from touching memory before this grid has
+// finished), then wait until the previous grid has completed and its writes
+// are visible.  Both are no-ops without programmatic dependent launch.
+__device__ __forceinline__ void pdl_entry() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- global memory
 
 // 16-byte streaming load: read-only path, no L1 allocation, 256-byte L2

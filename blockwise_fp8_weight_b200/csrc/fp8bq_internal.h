@@ -54,6 +54,30 @@ constexpr int kMaxDescTma = 128;    // 128 * (128 + 88) B + header = 27.7 KB
 static_assert(sizeof(DescPack<kMaxDescLarge>) < 32000, "kernel parameter limit");
 static_assert(sizeof(TmaPack<kMaxDescTma>) < 32000, "kernel parameter limit");
 
+// Programmatic dependent launch (on unless fp8bq_set_pdl(0)): every kernel of
+// the library is launched with programmatic stream serialization, so it may
+// be scheduled while the previous kernel of the stream drains; it lets the
+// next kernel launch at once and waits for the previous one (griddepcontrol)
+// before its first global-memory access.  Stream order of memory effects is
+// unchanged: only launch latency and the kernel prologue overlap.
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Kernel variants, by input element size and team shape.
 enum class Variant : int {
     Generic = 0,

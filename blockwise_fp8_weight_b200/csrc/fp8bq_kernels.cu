@@ -224,6 +224,7 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
+    dev::pdl_entry();
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
@@ -382,6 +383,7 @@ __device__ __forceinline__ float elem_f32(const char *p) {
 
 template <int ESIZE, int MAXD>
 __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPack<MAXD> p) {
+    dev::pdl_entry();
     const int lane = threadIdx.x & 31;
     const uint32_t stride = gridDim.x * 8;
     int d = 0;
@@ -414,6 +416,7 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
 // threads instead of 32.
 template <int ESIZE, int MAXD>
 __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ DescPack<MAXD> p) {
+    dev::pdl_entry();
     __shared__ uint32_t red[8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     int d = 0;
@@ -481,6 +484,7 @@ enum { MODE_ONE = 0, MODE_SUB = 1, MODE_CTA = 2 };
 template <int ESIZE, int STAGES, int MODE, int MAXD>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
     k_tma(const __grid_constant__ TmaPack<MAXD> P) {
+    dev::pdl_entry();
     constexpr int VEC = 16 / ESIZE;
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
     constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
@@ -705,6 +709,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
 template <int STAGES, int MAXD>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
     k_tma_pair(const __grid_constant__ TmaPack<MAXD> P) {
+    dev::pdl_entry();
     constexpr int ESIZE = 2, VEC = 8, BN = 128, BM = 128;
     constexpr int COLS = 2 * BN;                           // tile columns
     constexpr int STAGE_BYTES = BM * COLS * ESIZE;         // 64 KB
@@ -864,8 +869,7 @@ cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
     auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES>;
     static int occ = resident_ctas(kern, CTA, 0);
     const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
-    kern<<<grid, CTA, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, CTA, 0, st, p);
 }
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
@@ -900,24 +904,27 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
     // blocks of >= 2048 elements take one CTA each (the host groups generic
     // tensors by this size class, so it is uniform per launch)
     const bool cta = (int64_t)p.d[0].bm * p.d[0].bn >= 2048;
+    cudaError_t e;
     if (esize == 2) {
         if (cta) {
             static int occ = resident_ctas(k_generic_cta<2, MAXD>, 256, 0);
-            k_generic_cta<2, MAXD><<<grid_for(p.total_tiles, 1, occ), 256, 0, st>>>(p);
+            e = launch_kernel(k_generic_cta<2, MAXD>, grid_for(p.total_tiles, 1, occ), 256, 0, st,
+                              p);
         } else {
             static int occ = resident_ctas(k_generic<2, MAXD>, 256, 0);
-            k_generic<2, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+            e = launch_kernel(k_generic<2, MAXD>, grid_for(p.total_tiles, 8, occ), 256, 0, st, p);
         }
     } else {
         if (cta) {
             static int occ = resident_ctas(k_generic_cta<4, MAXD>, 256, 0);
-            k_generic_cta<4, MAXD><<<grid_for(p.total_tiles, 1, occ), 256, 0, st>>>(p);
+            e = launch_kernel(k_generic_cta<4, MAXD>, grid_for(p.total_tiles, 1, occ), 256, 0, st,
+                              p);
         } else {
             static int occ = resident_ctas(k_generic<4, MAXD>, 256, 0);
-            k_generic<4, MAXD><<<grid_for(p.total_tiles, 8, occ), 256, 0, st>>>(p);
+            e = launch_kernel(k_generic<4, MAXD>, grid_for(p.total_tiles, 8, occ), 256, 0, st, p);
         }
     }
-    return cudaGetLastError();
+    return e;
 }
 
 namespace {
@@ -929,8 +936,8 @@ cudaError_t launch_tma_t(const TmaPack<MAXD> &p, cudaStream_t st) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
     static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
-    kern<<<grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
+                         st, p);
 }
 }  // namespace
 
@@ -943,8 +950,8 @@ cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st) {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
     static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
-    kern<<<grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
+                         st, p);
 }
 
 template <int MAXD>

@@ -44,6 +44,7 @@ __device__ __forceinline__ void flush_max(uint32_t m, uint32_t *acc, int out, ui
 
 template <int ESIZE, int MAXD>
 __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ ScalePack<MAXD> p) {
+    dev::pdl_entry();
     constexpr int VEC = 16 / ESIZE;            // elements per 16-byte load
     constexpr int LOADS = kScaleItem / 256 / VEC;
     __shared__ uint32_t red[8];
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
 }
 
 __global__ void k_scale_finalize(float *scale_out, int n) {
+    dev::pdl_entry();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         const uint32_t bits = reinterpret_cast<const uint32_t *>(scale_out)[i];
         const float a = fmaxf(__uint_as_float(bits), kEps);
@@ -105,17 +107,13 @@ cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t 
     }
     const uint64_t cap = (uint64_t)sms * 8;
     const unsigned grid = (unsigned)(p.total < cap ? (p.total ? p.total : 1) : cap);
-    if (esize == 2)
-        k_scale_amax<2, MAXD><<<grid, 256, 0, st>>>(p);
-    else
-        k_scale_amax<4, MAXD><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    return esize == 2 ? launch_kernel(k_scale_amax<2, MAXD>, grid, 256, 0, st, p)
+                      : launch_kernel(k_scale_amax<4, MAXD>, grid, 256, 0, st, p);
 }
 
 cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st) {
     const int blocks = (n + 255) / 256;
-    k_scale_finalize<<<blocks < 1 ? 1 : blocks, 256, 0, st>>>(scale_out, n);
-    return cudaGetLastError();
+    return launch_kernel(k_scale_finalize, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n);
 }
 
 template cudaError_t launch_scale_amax<kMaxDescSmall>(const ScalePack<kMaxDescSmall> &, int,

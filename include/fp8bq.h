@@ -258,6 +258,22 @@ FP8BQ_API fp8bq_path fp8bq_get_path(void);
 FP8BQ_API int fp8bq_path_for(const fp8bq_desc *desc);
 
 /*
+ * Programmatic dependent launch (process-wide; on by default).  When on,
+ * every kernel of the library is launched so that it may be scheduled while
+ * the previous kernel of its stream is still finishing; each of its threads
+ * first waits (griddepcontrol.wait) until that kernel has completed and its
+ * writes are visible, so stream order of all memory effects is unchanged and
+ * only launch latency and the kernel prologue overlap.  The library's kernels
+ * also let the next kernel of the stream launch early; a kernel launched by
+ * the caller with programmatic stream serialization after one of ours must
+ * wait in the same way before it reads our outputs (as CUDA requires of any
+ * such kernel).  fp8bq_set_pdl(0) launches plainly; any other value turns it
+ * back on.  fp8bq_get_pdl returns 1 or 0.
+ */
+FP8BQ_API fp8bq_status fp8bq_set_pdl(int enable);
+FP8BQ_API int fp8bq_get_pdl(void);
+
+/*
  * Fault-injection and wait-limit knobs for tests (host side; process-wide).
  * fp8bq_debug_set_wait_limit_ns bounds every device-side wait of the TMA
  * kernel (default 2e9 ns; 0 restores the default).

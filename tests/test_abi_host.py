@@ -185,6 +185,17 @@ def test_variant_choice(path_guard):
     assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_GENERIC
 
 
+def test_pdl_switch():
+    assert fq.fp8bq_get_pdl() == 1                       # on by default
+    try:
+        assert fq.fp8bq_set_pdl(0) == fq.FP8BQ_OK
+        assert fq.fp8bq_get_pdl() == 0
+        assert fq.fp8bq_set_pdl(5) == fq.FP8BQ_OK
+        assert fq.fp8bq_get_pdl() == 1
+    finally:
+        fq.fp8bq_set_pdl(1)
+
+
 def test_debug_knobs():
     assert fq.fp8bq_debug_set_inject(2) == fq.FP8BQ_ERR_ARG
     assert fq.fp8bq_debug_set_inject(0) == fq.FP8BQ_OK
