@@ -106,6 +106,7 @@ def aggregate(bytes_per_step: int, steps: int, world: int, max_elapsed_s: float)
 
 
 def workload(name: str):
+    from synth import TensorSpec
     from synth import workloads as W
     if name == "qwen3_8b_model":
         return W.qwen3_8b_model(), ("Qwen3-8B-shaped full weight set: 36 layers x (q,k,v,o,"
@@ -134,6 +135,13 @@ def workload(name: str):
         return W.edge(), ("ragged and small-block edge set in one grouped call: bf16 and fp32 "
                           "4000x4100, 130x129, 1x128, 12345x4096, 4000x4100 with ld 4164 "
                           "(block 128x128), bf16 16384x4096 with [1,128] and [64,64] blocks")
+    if name.startswith("shape:"):  # shape:[BATCHx]MxN[:f32] -- one tensor, block 128x128
+        dims, _, dt = name[6:].partition(":")
+        v = [int(t) for t in dims.split("x")]
+        batch, M, N = (v if len(v) == 3 else [1] + v)
+        sp = TensorSpec(f"shape.{dims}", M, N, batch=batch, dtype=dt or "bf16", seed=5,
+                        tensor_id=0, sigma=0.02)
+        return [sp], f"one {sp.dtype} tensor [{batch}, {M}, {N}], block 128x128, N(0, 0.02)"
     if name in ("act_1x128", "blk_64x64"):
         sp = [t for t in W.edge() if t.name.endswith("b1x128" if name == "act_1x128" else "b64x64")]
         return sp, f"bf16 16384x4096, N(0,1) x row lognormal(0,1), blocks {sp[0].block}"
@@ -431,6 +439,12 @@ def run_ours(args) -> None:
     dev = torch.device("cuda", local_rank)
     dist = Dist(world, "nccl", dev)
     specs, wl_desc = workload(args.workload)
+    if args.only:  # a subset of the workload's tensors (by name)
+        import re
+        specs = [sp for sp in specs if re.search(args.only, sp.name)]
+        if not specs:
+            raise SystemExit(f"--only {args.only!r} matches no tensor of {args.workload}")
+        wl_desc += f"; only the tensors matching {args.only!r}"
     if args.repeat > 1:  # the same tensor list args.repeat times, fresh values each time
         import dataclasses
         specs = [dataclasses.replace(sp, name=f"{sp.name}.r{k}", tensor_id=sp.tensor_id + 4096 * k,
@@ -771,13 +785,15 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen3_8b_model",
-                    choices=["qwen3_8b_model", "qwen3_8b_layer", "moe_layer", "small",
-                             "act_1x128", "blk_64x64", "qkv", "ragged", "edge",
-                             "qwen3_8b_layer_f32"])
+                    help="qwen3_8b_model (default), qwen3_8b_layer, qwen3_8b_layer_f32, "
+                         "moe_layer, small, act_1x128, blk_64x64, qkv, ragged, edge, or "
+                         "shape:[BATCHx]MxN[:f32] for one tensor of that shape")
     ap.add_argument("--path", choices=list(PATHS), default="auto")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--repeat", type=int, default=1,
                     help="replicate the workload's tensor list this many times (distinct values)")
+    ap.add_argument("--only", default=None, metavar="REGEX",
+                    help="keep only the workload's tensors whose name matches REGEX")
     ap.add_argument("--pdl", choices=["on", "off"], default="on",
                     help="programmatic dependent launch of the library's kernels")
     ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",

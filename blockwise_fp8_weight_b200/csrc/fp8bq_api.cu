@@ -393,12 +393,15 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
     size_t i = 0;
     while (i < idx.size()) {
         pack_header(P.p);
+        P.evict_first = 0;
         while (i < idx.size() && P.p.n < MAXD) {
             const fp8bq_desc &D = t[idx[i]];
             const uint64_t tiles = tiles_of(D, Variant::Tma);
             if (P.p.n > 0 && (uint64_t)P.p.total_tiles + tiles >= (1ull << 31)) break;
             fill_tile_desc(D, Variant::Tma, P.p.total_tiles, &P.p.d[P.p.n]);
             P.maps[P.p.n] = maps[i];
+            const uint64_t in_bytes = (uint64_t)D.batch * (uint64_t)D.M * (uint64_t)D.N * es;
+            if (in_bytes >= kEvictFirstMinBytes) P.evict_first = 1;
             P.p.total_tiles += (uint32_t)tiles;
             ++P.p.n;
             ++i;

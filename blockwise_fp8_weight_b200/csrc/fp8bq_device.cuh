@@ -190,13 +190,26 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
 }
 
 // 3-D TMA tile load into shared memory, completing on `bar` (no multicast).
+// evict_first: the tile's lines get an L2 evict-first policy (every input
+// byte is read once); otherwise the default priority.
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar,
-                                            int c0, int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(smem_dst)),
-        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
-        : "memory");
+                                            int c0, int c1, int c2, bool evict_first) {
+    if (evict_first) {  // a compile-time constant at every call
+        asm volatile(
+            "{\n\t.reg .b64 pol;\n\t"
+            "createpolicy.fractional.L2::evict_first.b64 pol, 1.0;\n\t"
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], pol;\n\t}" ::"r"(
+                smem_addr(smem_dst)),
+            "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+            : "memory");
+    } else {
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(smem_dst)),
+            "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+            : "memory");
+    }
 }
 
 // Named barrier over `count` threads.

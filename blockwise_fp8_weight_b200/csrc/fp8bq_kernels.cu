@@ -481,7 +481,7 @@ struct TileWalk {
 //             reduced within its group of L lanes with shuffles.
 enum { MODE_ONE = 0, MODE_SUB = 1, MODE_CTA = 2 };
 
-template <int ESIZE, int STAGES, int MODE, int MAXD>
+template <int ESIZE, int STAGES, int MODE, int MAXD, bool EF>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
     k_tma(const __grid_constant__ TmaPack<MAXD> P) {
     dev::pdl_entry();
@@ -547,7 +547,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                 dropped0 = true;  // fault injection: this slot's barrier can never complete
             else
                 dev::tma_load_3d(ring + (size_t)st * STAGE_BYTES, &P.maps[d], &full[st],
-                                 T.bj * bn, T.bi * bm, T.b);
+                                 T.bj * bn, T.bi * bm, T.b, EF);
         }
         // Drain: each slot's last issued copy must land before the CTA exits.
         const uint32_t issued = k;
@@ -706,7 +706,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
 #define FP8BQ_TMA_PAIR_STAGES 2   // 64 KB ring slots (3 measured 12 % slower)
 #endif
 
-template <int STAGES, int MAXD>
+template <int STAGES, int MAXD, bool EF>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
     k_tma_pair(const __grid_constant__ TmaPack<MAXD> P) {
     dev::pdl_entry();
@@ -769,7 +769,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
                 dropped0 = true;
             else
                 dev::tma_load_3d(ring + (size_t)st * STAGE_BYTES, &P.maps[d], &full[st],
-                                 T.bj * BN, T.bi * BM, T.b);
+                                 T.bj * BN, T.bi * BM, T.b, EF);
         }
         const uint32_t issued = k;
         for (int st = 0; st < STAGES && (uint32_t)st < issued; ++st) {
@@ -928,10 +928,31 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
 }
 
 namespace {
+template <int ESIZE, int STAGES, int MODE, int MAXD, bool EF>
+cudaError_t launch_tma_e(const TmaPack<MAXD> &p, cudaStream_t st) {
+    constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
+    auto kern = k_tma<ESIZE, STAGES, MODE, MAXD, EF>;
+    static cudaError_t attr =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (attr != cudaSuccess) return attr;
+    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
+                         st, p);
+}
+
+// The L2 policy of the tile loads is a template parameter, so the default
+// kernels carry no trace of the other policy.
 template <int ESIZE, int STAGES, int MODE, int MAXD>
 cudaError_t launch_tma_t(const TmaPack<MAXD> &p, cudaStream_t st) {
-    constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
-    auto kern = k_tma<ESIZE, STAGES, MODE, MAXD>;
+    return p.evict_first ? launch_tma_e<ESIZE, STAGES, MODE, MAXD, true>(p, st)
+                         : launch_tma_e<ESIZE, STAGES, MODE, MAXD, false>(p, st);
+}
+
+template <int MAXD, bool EF>
+cudaError_t launch_tma_pair_e(const TmaPack<MAXD> &p, cudaStream_t st) {
+    constexpr int S = FP8BQ_TMA_PAIR_STAGES;
+    constexpr size_t smem = (size_t)S * 128 * 256 * 2;
+    auto kern = k_tma_pair<S, MAXD, EF>;
     static cudaError_t attr =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (attr != cudaSuccess) return attr;
@@ -943,15 +964,8 @@ cudaError_t launch_tma_t(const TmaPack<MAXD> &p, cudaStream_t st) {
 
 template <int MAXD>
 cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st) {
-    constexpr int S = FP8BQ_TMA_PAIR_STAGES;
-    constexpr size_t smem = (size_t)S * 128 * 256 * 2;
-    auto kern = k_tma_pair<S, MAXD>;
-    static cudaError_t attr =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (attr != cudaSuccess) return attr;
-    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
-                         st, p);
+    return p.evict_first ? launch_tma_pair_e<MAXD, true>(p, st)
+                         : launch_tma_pair_e<MAXD, false>(p, st);
 }
 
 template <int MAXD>
