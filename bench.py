@@ -774,8 +774,8 @@ def run_scale_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc) -> No
                        "bytes_per_step": nbytes, "tensors": len(specs)},
             "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
                          "frac": value / world / peak, "traffic": None, "peak_source": kind,
-                         "note": "one memset, one grid-wide pass and one finalize launch per step"},
-            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}), flush=True)
+                         "note": "one zeroing, one grid-wide pass and one finalize launch per step"},
+            "gpu_launches": 3 * args.steps, "clocks": clk.summary()}), flush=True)
 
 
 def main() -> None:

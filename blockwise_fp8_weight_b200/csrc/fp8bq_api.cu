@@ -668,7 +668,7 @@ fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out
     }
     const fp8bq_status sd = check_device();
     if (sd != FP8BQ_OK) return sd;
-    if (cudaMemsetAsync(scale_out, 0, (size_t)n * 4, stream) != cudaSuccess) {
+    if (launch_scale_zero(scale_out, n, stream) != cudaSuccess) {
         cudaGetLastError();
         return FP8BQ_ERR_DEVICE;
     }

@@ -161,6 +161,7 @@ struct ScalePack {
 static_assert(sizeof(ScalePack<kMaxDescLarge>) < 32000, "kernel parameter limit");
 template <int MAXD>
 cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t st);
+cudaError_t launch_scale_zero(float *scale_out, int n, cudaStream_t st);
 cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st);
 
 // Device error word access (fp8bq_kernels.cu).

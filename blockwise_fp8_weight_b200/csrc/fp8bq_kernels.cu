@@ -35,6 +35,16 @@ constexpr uint64_t kDrainLimitNs = 2000000000ull;
 #ifndef FP8BQ_VEC_CTAS_PER_SM
 #define FP8BQ_VEC_CTAS_PER_SM 2   // resident 256-thread vector CTAs per SM
 #endif
+// Depth of the vector kernel's cp.async ring (16-byte aligned rows), by team.
+// Measured on B200 (stages 0 = register ping-pong / 2 / 3 / 4): [1,128] blocks
+// 4.95 / 5.37 / 5.47 / 4.46 TB/s; [64,64] blocks 5.57 / 6.21 / 6.03 / 5.39;
+// 128x128 blocks 5.63 / 6.22 / 6.20 / 5.23 (4 stages leave one CTA per SM).
+#ifndef FP8BQ_VEC_STAGES_T16
+#define FP8BQ_VEC_STAGES_T16 3
+#endif
+#ifndef FP8BQ_VEC_STAGES
+#define FP8BQ_VEC_STAGES 2
+#endif
 #ifndef FP8BQ_TMA_STAGES_BF16
 #define FP8BQ_TMA_STAGES_BF16 4   // 32 KB ring slots per TMA CTA (bf16 tiles)
 #endif
@@ -211,7 +221,11 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // team holds the vectors (row0 + i * rstep, cv), i < V, with cv = lane % vpr,
 // row0 = lane / vpr, rstep = TEAM / vpr: consecutive lanes read consecutive
 // 16-byte pieces of a row, so each warp load covers whole 256-byte row
-// segments.  bm and bn are the same for every tensor of a launch.
+// segments.  bm and bn are the same for every tensor of a launch.  The tile's
+// vectors reach the registers through a per-thread cp.async ring in shared
+// memory (S stages), or, for 8-byte-aligned rows, by direct loads with the
+// next tile loaded into a second register set while the current one is
+// reduced and stored.
 
 //
 // G > 1 (small blocks): a tile is G vertically adjacent blocks and slot i of
@@ -221,11 +235,16 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // HALVES (rows only 8-byte aligned; N a multiple of VEC / 2): the same
 // geometry, each 16-byte vector moved as two 8-byte halves; a half beyond
 // the row end reads as zeros (no effect on the absmax) and is not stored.
-template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
+//
+// S > 0 (16-byte aligned rows only): the loads go through a private ring of S
+// stages per thread in shared memory (cp.async), S - 1 tiles in flight while
+// one is reduced and stored.
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, int S>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     dev::pdl_entry();
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
+    static_assert(!(HALVES && S > 0), "the cp.async ring takes 16-byte vectors only");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -332,6 +351,59 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         }
         if (lane == 0) *T.sdst = s;
     };
+
+    if constexpr (S > 0) {
+        extern __shared__ __align__(1024) uint8_t ring[];  // dynamic shared memory
+        uint4 *const stage = reinterpret_cast<uint4 *>(ring);  // [S][V][CTA] 16-byte vectors
+        auto issue = [&](int s, const Tile &T) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int r = row0 + i * rstep;
+                const bool ok = r < T.rows && colv < T.cols;
+                const char *src = ok ? T.src + ((int64_t)r * T.ld + colv) * ESIZE : T.src;
+                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], src, ok);
+            }
+            dev::cp_async_commit();
+        };
+        Tile Ts[S];
+        uint32_t tn = t;  // next tile to issue; t: next tile to process
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            if (tn < p.total_tiles) {
+                Ts[s] = make_tile<ESIZE, G>(p, tn, d);
+                issue(s, Ts[s]);
+            } else {
+                dev::cp_async_commit();  // empty group: keeps the wait count uniform
+            }
+            tn += stride;
+        }
+        uint32_t it = 0;
+        bool more = true;
+        while (more) {
+#pragma unroll
+            for (int s = 0; s < S; ++s) {
+                if (t >= p.total_tiles) {
+                    more = false;
+                    break;
+                }
+                dev::cp_async_wait<S - 1>();  // this thread's copies of stage s have landed
+                uint4 R[V];
+#pragma unroll
+                for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
+                process(R, Ts[s], it++);  // consumes R: the stage is free again
+                if (tn < p.total_tiles) {
+                    Ts[s] = make_tile<ESIZE, G>(p, tn, d);
+                    issue(s, Ts[s]);
+                } else {
+                    dev::cp_async_commit();
+                }
+                tn += stride;
+                t += stride;
+            }
+        }
+        dev::cp_async_wait<0>();
+        return;
+    }
 
     uint4 A[V], B[V];
     Tile ta = make_tile<ESIZE, G>(p, t, d);
@@ -866,10 +938,17 @@ unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
-    auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES>;
-    static int occ = resident_ctas(kern, CTA, 0);
+    constexpr int S = HALVES ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
+    constexpr size_t smem = (size_t)S * V * CTA * 16;
+    auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES, S>;
+    if constexpr (smem > 48 * 1024) {
+        static cudaError_t attr =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (attr != cudaSuccess) return attr;
+    }
+    static int occ = resident_ctas(kern, CTA, smem);
     const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
-    return launch_kernel(kern, grid, CTA, 0, st, p);
+    return launch_kernel(kern, grid, CTA, smem, st, p);
 }
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>

@@ -85,6 +85,14 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
     if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red);
 }
 
+// Zero the accumulators (a kernel rather than a memset, so that the next
+// kernel of the chain can overlap its launch with this one).
+__global__ void k_scale_zero(float *scale_out, int n) {
+    dev::pdl_entry();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+        scale_out[i] = 0.0f;
+}
+
 __global__ void k_scale_finalize(float *scale_out, int n) {
     dev::pdl_entry();
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -109,6 +117,11 @@ cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t 
     const unsigned grid = (unsigned)(p.total < cap ? (p.total ? p.total : 1) : cap);
     return esize == 2 ? launch_kernel(k_scale_amax<2, MAXD>, grid, 256, 0, st, p)
                       : launch_kernel(k_scale_amax<4, MAXD>, grid, 256, 0, st, p);
+}
+
+cudaError_t launch_scale_zero(float *scale_out, int n, cudaStream_t st) {
+    const int blocks = (n + 255) / 256;
+    return launch_kernel(k_scale_zero, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n);
 }
 
 cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st) {

@@ -47,7 +47,7 @@ def test_chain_keeps_stream_order(pdl):
             y, s = fq.scaled_fp8_blockwise(x, [128, 128])     # ours reads it
             z = fq.dequantize_fp8_blockwise(y, s)             # ours reads ours
             zmax = z.float().abs().amax()                     # PyTorch reads ours
-            sc = fq.tensor_scales([x])                        # memset, then two kernels
+            sc = fq.tensor_scales([x])                        # zero, amax, finalize kernels
             outs.append((y, s, z, zmax, sc))
         torch.cuda.synchronize()
     finally:
