@@ -223,9 +223,7 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // 16-byte pieces of a row, so each warp load covers whole 256-byte row
 // segments.  bm and bn are the same for every tensor of a launch.  The tile's
 // vectors reach the registers through a per-thread cp.async ring in shared
-// memory (S stages), or, for 8-byte-aligned rows, by direct loads with the
-// next tile loaded into a second register set while the current one is
-// reduced and stored.
+// memory (S stages).
 
 //
 // G > 1 (small blocks): a tile is G vertically adjacent blocks and slot i of
@@ -236,15 +234,15 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // geometry, each 16-byte vector moved as two 8-byte halves; a half beyond
 // the row end reads as zeros (no effect on the absmax) and is not stored.
 //
-// S > 0 (16-byte aligned rows only): the loads go through a private ring of S
-// stages per thread in shared memory (cp.async), S - 1 tiles in flight while
-// one is reduced and stored.
+// S > 0: the loads go through a private ring of S stages per thread in shared
+// memory (cp.async; two 8-byte copies per vector in HALVES mode), S - 1 tiles
+// in flight while one is reduced and stored.  S == 0: two register sets, the
+// next tile loaded while the current one is processed.
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, int S>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     dev::pdl_entry();
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
-    static_assert(!(HALVES && S > 0), "the cp.async ring takes 16-byte vectors only");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -361,7 +359,15 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
                 const int r = row0 + i * rstep;
                 const bool ok = r < T.rows && colv < T.cols;
                 const char *src = ok ? T.src + ((int64_t)r * T.ld + colv) * ESIZE : T.src;
-                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], src, ok);
+                uint4 *dst = &stage[(s * V + i) * CTA + threadIdx.x];
+                if constexpr (HALVES) {
+                    const bool ok_hi = ok && hi_ok(T);
+                    dev::cp_async_8(dst, src, ok);
+                    dev::cp_async_8(reinterpret_cast<char *>(dst) + 8, ok_hi ? src + 8 : src,
+                                    ok_hi);
+                } else {
+                    dev::cp_async_16(dst, src, ok);
+                }
             }
             dev::cp_async_commit();
         };
@@ -938,7 +944,7 @@ unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
-    constexpr int S = HALVES ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
+    constexpr int S = TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
     constexpr size_t smem = (size_t)S * V * CTA * 16;
     auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES, S>;
     if constexpr (smem > 48 * 1024) {
