@@ -51,7 +51,9 @@ if ROOT not in sys.path:
 
 METRIC = "blockwise FP8 quant GB/s (bytes in+out) and % of B200 HBM peak, 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["blockwise_fp8_weight_b200/csrc/fp8bq_kernels.cu",
+# the sources of the TMA kernels, whose DRAM traffic profiles/traffic.txt records
+KERNEL_SOURCES = ["blockwise_fp8_weight_b200/csrc/fp8bq_tma.cu",
+                  "blockwise_fp8_weight_b200/csrc/fp8bq_tile.cuh",
                   "blockwise_fp8_weight_b200/csrc/fp8bq_device.cuh",
                   "blockwise_fp8_weight_b200/csrc/fp8bq_internal.h"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.txt")

@@ -16,9 +16,10 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(CSRC, f) for f in ("fp8bq_api.cu", "fp8bq_kernels.cu", "fp8bq_dequant.cu",
-                                                   "fp8bq_scale.cu")]
-HEADERS = [os.path.join(CSRC, f) for f in ("fp8bq_internal.h", "fp8bq_device.cuh")] + [
+SOURCES = [os.path.join(CSRC, f) for f in ("fp8bq_api.cu", "fp8bq_kernels.cu", "fp8bq_tma.cu",
+                                                   "fp8bq_dequant.cu", "fp8bq_scale.cu")]
+HEADERS = [os.path.join(CSRC, f) for f in ("fp8bq_internal.h", "fp8bq_device.cuh",
+                                                   "fp8bq_tile.cuh")] + [
     os.path.join(ROOT, "include", "fp8bq.h")]
 LIB = os.path.join(PKG, "libfp8bq.so")
 

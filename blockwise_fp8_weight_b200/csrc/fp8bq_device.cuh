@@ -150,13 +150,6 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *src, boo
                  "l"(src), "r"(ok ? 16 : 0)
                  : "memory");
 }
-// The same for 8 bytes (through L1: the two halves of a 16-byte vector are
-// copied by two such copies).
-__device__ __forceinline__ void cp_async_8(void *smem_dst, const void *src, bool ok) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_addr(smem_dst)),
-                 "l"(src), "r"(ok ? 8 : 0)
-                 : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }

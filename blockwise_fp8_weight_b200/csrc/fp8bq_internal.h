@@ -97,7 +97,8 @@ enum class Variant : int {
     Tma = 4,
 };
 
-// Launchers (fp8bq_kernels.cu).  Each returns cudaSuccess or the launch error.
+// Launchers (vector and generic: fp8bq_kernels.cu; TMA: fp8bq_tma.cu).  Each
+// returns cudaSuccess or the launch error.
 // halves: rows only 8-byte aligned (each 16-byte vector moved as two halves)
 template <int MAXD>
 cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
@@ -164,7 +165,7 @@ cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t 
 cudaError_t launch_scale_zero(float *scale_out, int n, cudaStream_t st);
 cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st);
 
-// Device error word access (fp8bq_kernels.cu).
+// Device error word access (fp8bq_tma.cu).
 cudaError_t read_and_clear_error_word(uint32_t *out);
 
 // Team geometry used by the vector kernels (host eligibility must agree).
