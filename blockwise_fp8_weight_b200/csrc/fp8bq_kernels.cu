@@ -15,7 +15,8 @@
 // all tensors of a group (the descriptor table travels in the kernel
 // parameters); three variants share the arithmetic:
 //   k_vector   16-byte coalesced vectors staged through a per-thread cp.async
-//              ring (this file);
+//              ring (rows only 8-byte aligned: two 8-byte loads per vector
+//              straight into registers) (this file);
 //   k_tma      a producer warp streams 3-D TMA tiles into a shared-memory
 //              ring, consumer warps reduce and quantize (fp8bq_tma.cu);
 //   k_generic  element-wise loads, one warp per block: any alignment,
@@ -65,8 +66,8 @@ __device__ __forceinline__ uint32_t reduce_scatter8x16(const uint32_t (&m)[8], u
     return max(c, __shfl_xor_sync(mask, c, 1));
 }
 
-// The same for a lane's 16 bytes held as two 8-byte halves (rows that are
-// only 8-byte aligned): each half is quantized and stored on its own, the
+// vec_quant_store for a lane's 16 bytes held as two 8-byte halves (rows that
+// are only 8-byte aligned): each half is quantized and stored on its own, the
 // upper one only when hi_ok (it lies inside the row).  Codes: 4 bytes per
 // bf16 half, 2 per fp32 half.
 template <int ESIZE>
