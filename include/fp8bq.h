@@ -32,6 +32,11 @@
  * the current device).  The library writes only y and descale, allocates no
  * device memory per call, and keeps no pointer after a call returns.
  *
+ * Devices: a process drives one GPU (one process per GPU, as under torchrun).
+ * The library raises its kernels' dynamic shared-memory limit, and sizes
+ * their grids, on the first device that launches them; calls made later on
+ * another device of the same process are not supported.
+ *
  * Execution: calls are asynchronous on `stream`, like a kernel launch.  All
  * arguments are checked before anything is launched: a call that returns an
  * argument error (anything but FP8BQ_ERR_DEVICE) launched nothing.  A call may
