@@ -257,6 +257,17 @@ def check(status: int, what: str = "") -> None:
 # ----------------------------------------------------------------- PyTorch conveniences
 
 
+def _check_cuda(t, what: str) -> None:
+    """The library reads and writes device memory of the current device: refuse
+    anything else here, before a kernel could touch a host address."""
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{what} is on {t.device}, not on the current device cuda:{cur}")
+
+
 def _dtype_code(t) -> int:
     import torch
     if t.dtype == torch.bfloat16:
@@ -272,6 +283,9 @@ def make_desc(x, y, s, block=DEFAULT_BLOCK) -> fp8bq_desc:
     descale ``s`` (contiguous [(E,) ceil(M/bm), ceil(N/bn)])."""
     if x.dim() not in (2, 3):
         raise ValueError("expected a 2-D weight or a 3-D stack of expert weights")
+    _check_cuda(x, "the input")
+    _check_cuda(y, "the e4m3fn output")
+    _check_cuda(s, "the descale output")
     if x.shape[-1] > 1 and x.stride(-1) != 1:
         raise ValueError("the last dimension of the input must have unit stride")
     d = fp8bq_desc()
@@ -307,6 +321,7 @@ def scaled_fp8_blockwise(data_hp, weight_block_size=DEFAULT_BLOCK, stream=None):
     fp32 (the "weight_scale_inv" of the rollout engine).
     """
     block = tuple(int(b) for b in weight_block_size)
+    _check_cuda(data_hp, "data_hp")
     y, s = _outputs(data_hp, block)
     check(fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream),
           "scaled_fp8_blockwise")
@@ -321,6 +336,8 @@ def dequantize_fp8_blockwise(fp8_data, descale, weight_block_size=DEFAULT_BLOCK,
     out_dtype = torch.bfloat16 if out_dtype is None else out_dtype
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise TypeError("out_dtype must be torch.bfloat16 or torch.float32")
+    _check_cuda(fp8_data, "fp8_data")
+    _check_cuda(descale, "descale")
     if not fp8_data.is_contiguous() or not descale.is_contiguous():
         raise ValueError("fp8_data and descale must be contiguous")
     bm, bn = (int(b) for b in weight_block_size)
@@ -341,9 +358,11 @@ def tensor_scales(tensors, stream=None):
     tensors = list(tensors)
     if not tensors:
         raise ValueError("no tensors")
+    _check_cuda(tensors[0], "every tensor")
     out = torch.empty(len(tensors), dtype=torch.float32, device=tensors[0].device)
     descs = []
     for t in tensors:
+        _check_cuda(t, "every tensor")
         if not t.is_contiguous():
             raise ValueError("tensors must be contiguous")
         d = fp8bq_scale_desc()
@@ -360,6 +379,7 @@ def quant_weights(weights: Iterable, weight_block_size=DEFAULT_BLOCK, stream=Non
     block = tuple(int(b) for b in weight_block_size)
     items, descs = [], []
     for name, w in weights:
+        _check_cuda(w, name)
         y, s = _outputs(w, block)
         items.append((name, y, s, w))
         descs.append(make_desc(w, y, s, block))

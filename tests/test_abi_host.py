@@ -291,3 +291,22 @@ def test_tensor_scale_argument_errors():
     assert T([sdesc(x=S - 100)]) == fq.FP8BQ_ERR_OVERLAP
     if NO_GPU:
         assert T([sdesc(), sdesc(x=0, numel=0)]) == fq.FP8BQ_ERR_DEVICE
+
+
+def test_conveniences_refuse_host_tensors():
+    """The PyTorch conveniences hand only device memory of the current device
+    to the library: host tensors are refused before any call into it."""
+    import torch
+    w = torch.zeros(256, 384, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.scaled_fp8_blockwise(w)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.quant_weights([("layers.0.q_proj.weight", w)])
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.tensor_scales([w])
+    y = torch.zeros(256, 384, dtype=torch.uint8)
+    s = torch.zeros(2, 3, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.dequantize_fp8_blockwise(y, s)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        fq.make_desc(w, y, s)
