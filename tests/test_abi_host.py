@@ -310,3 +310,25 @@ def test_conveniences_refuse_host_tensors():
         fq.dequantize_fp8_blockwise(y, s)
     with pytest.raises(ValueError, match="CUDA tensor"):
         fq.make_desc(w, y, s)
+
+
+def test_c_consumer_compiles_links_and_runs(tmp_path):
+    """tests/c/abi_consumer.c: the header is C99, every declared entry point
+    links from plain C, the descriptor sizes are the documented ones, and the
+    device-free calls behave as documented."""
+    import shutil
+    import subprocess
+    from blockwise_fp8_weight_b200 import build as B
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    fq.lib()  # builds the library if needed
+    cuda_inc = os.path.join(os.path.dirname(os.path.dirname(os.path.realpath(B.nvcc()))), "include")
+    exe = str(tmp_path / "abi_consumer")
+    pkg = os.path.dirname(fq.LIB_PATH)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", cuda_inc, os.path.join(ROOT, "tests", "c", "abi_consumer.c"), "-L", pkg,
+                    "-lfp8bq", f"-Wl,-rpath,{pkg}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert "abi consumer ok" in r.stdout
