@@ -199,8 +199,9 @@ bool tma_geom(const fp8bq_desc &D, int *group, bool *subwarp) {
 
 // AUTO: the TMA ring when one block fills a ring slot of at least 16 KB
 // (measured: with stacked small blocks the ring's 8 consumer warps spend too
-// long per tile, and the register-tile vector kernel is 2-2.5x faster), the
-// vector kernel for other aligned tensors, the generic kernel otherwise.
+// long per tile, and the team-per-tile vector kernel is 2-2.5x faster), the
+// vector kernel for other 16- or 8-byte-aligned tensors, the generic kernel
+// otherwise.
 constexpr int64_t kTmaMinSlotBytes = 16384;
 
 Variant choose(const fp8bq_desc &D, int path) {
@@ -231,7 +232,7 @@ bool tma_paired(const fp8bq_desc &D) {
 // ------------------------------------------------------------------ tensor maps
 
 // L2 promotion of the TMA tile loads (CUtensorMapL2promotion: 0 none, 1 64 B,
-// 2 128 B, 3 256 B); a tile row is 256 bytes of bf16.
+// 2 128 B, 3 256 B); a block row is 256 bytes of bf16 (512 in a paired tile).
 #ifndef FP8BQ_TMA_L2_PROMOTION
 #define FP8BQ_TMA_L2_PROMOTION 3
 #endif
