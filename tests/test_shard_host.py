@@ -64,7 +64,13 @@ def _rank(rank, world, port, case, q):
         fy, fs = gather_quantized_shards(torch.from_numpy(y), torch.from_numpy(s), M, N, block)
         wy, ws = oracle.quantize(np.ascontiguousarray(x), M, N, N, *block)
         ok = (fy.shape == (M, N) and np.array_equal(fy.numpy(), wy)
-              and np.array_equal(fs.numpy().view(np.uint32), ws.view(np.uint32)))
+              and np.array_equal(fs.numpy().view(np.uint32), ws.view(np.uint32))
+              # the results are the leading rows of the (padded) gather
+              # buffers, not copies
+              and fy.untyped_storage().nbytes() > fy.numel()
+              and fy.data_ptr() == fy.untyped_storage().data_ptr()
+              and fs.data_ptr() == fs.untyped_storage().data_ptr()
+              and fy.is_contiguous() and fs.is_contiguous())
         q.put((rank, ok))
     finally:
         dist.destroy_process_group()
