@@ -5,7 +5,7 @@
                     [--workload qwen3_8b_model|qwen3_8b_layer|qwen3_8b_layer_f32|moe_layer|
                                 small|act_1x128|blk_64x64|qkv|ragged|edge] [--repeat R]
                     [--path auto|vector|tma|generic] [--mode grouped|per_layer|per_tensor]
-                    [--op quantize|dequantize|tensor_scale] [--pdl on|off]
+                    [--op quantize|dequantize|tensor_scale|shard] [--pdl on|off]
 
 A step is one pass of the whole quantizer over the workload: by default the
 full Qwen3-8B-shaped weight set (36 layers x q,k,v,o,gate,up,down = 252 bf16
@@ -299,20 +299,21 @@ def kernel_digest() -> str:
 
 
 def traffic_for(workload_name: str, path: str, launches: int):
-    """DRAM bytes per launch, from the committed ncu record of this workload
-    (profiles/traffic.txt: "<workload> <path> <kernel sources sha256/16>
-    <dram bytes per step>"), if it was taken on the current kernel sources;
-    else None."""
+    """(DRAM bytes per launch, how they were obtained) from the committed ncu
+    record of this workload (profiles/traffic.txt: "<workload> <path> <kernel
+    sources sha256/16> <dram bytes per step> <source>", the source saying
+    whether the step was captured or scaled from a smaller case), if it was
+    taken on the current kernel sources; else (None, None)."""
     try:
         lines = open(TRAFFIC_FILE).read().splitlines()
     except OSError:
-        return None
+        return None, None
     for line in lines:
-        f = line.split()
-        if len(f) == 4 and not line.startswith("#") and f[0] == workload_name and f[1] == path \
+        f = line.split(maxsplit=4)
+        if len(f) >= 4 and not line.startswith("#") and f[0] == workload_name and f[1] == path \
                 and f[2] == kernel_digest():
-            return float(f[3]) / max(launches, 1)
-    return None
+            return float(f[3]) / max(launches, 1), (f[4] if len(f) > 4 else "captured")
+    return None, None
 
 
 # ------------------------------------------------------------------ arms
@@ -518,9 +519,11 @@ def run_ours(args) -> None:
     max_elapsed = dist.max(elapsed_s)
     value = aggregate(bytes_per_step, args.steps, world, max_elapsed)
 
-    if args.op in ("dequantize", "tensor_scale"):
+    if args.op in ("dequantize", "tensor_scale", "shard"):
         if args.op == "dequantize":
             run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_desc)
+        elif args.op == "shard":
+            run_shard_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc)
         else:
             run_scale_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc)
         fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
@@ -610,7 +613,7 @@ def run_ours(args) -> None:
     l2_mb = torch.cuda.get_device_properties(dev).L2_cache_size / 1e6
     launch_s = elapsed_s / args.steps / max(launches, 1)
     achieved = bytes_per_step / max(launches, 1) / launch_s / 1e9
-    traffic = traffic_for(args.workload, args.path, launches)
+    traffic, traffic_source = traffic_for(args.workload, args.path, launches)
 
     if rank == 0:
         line = {
@@ -631,6 +634,7 @@ def run_ours(args) -> None:
                        "elements_per_s": elements * args.steps * world / max_elapsed},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         "traffic_source": traffic_source,
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                          if peak_kind == "measured" else "fallback 6650 GB/s",
                          "kernel_launches_per_step": launches,
@@ -726,6 +730,117 @@ def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_de
               flush=True)
 
 
+def run_shard_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc) -> None:
+    """Time the weight sync of row-sharded weights two ways, every rank holding
+    its block-row shard of every (2-D) weight of the workload:
+      ours      one grouped quantize launch writes every shard's codes and
+                descales into its slot of the gather buffers, then each
+                weight's codes and descales are all-gathered in place;
+      baseline  each weight's bf16 shards are all-gathered, then the whole
+                weights are quantized (one grouped launch).
+    Value: ours, in GB/s of the quantizer's algorithmic bytes of the whole
+    weights (the same bytes as the default metric)."""
+    import socket
+
+    import torch
+    import torch.distributed as tdist
+    import blockwise_fp8_weight_b200 as fq
+    from blockwise_fp8_weight_b200.shard import ShardedQuantGather, shard_rows
+    if not tdist.is_initialized():  # one rank: a one-process NCCL group
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        tdist.init_process_group("nccl", store=tdist.TCPStore("127.0.0.1", port, 1, True),
+                                 rank=0, world_size=1, device_id=dev)
+    idx = [i for i, sp in enumerate(specs) if sp.batch == 1 and sp.row_stride == sp.N
+           and sp.dtype == "bf16"]
+    if not idx:
+        raise SystemExit("--op shard needs 2-D bf16 tensors without row padding")
+    bm, bn = specs[idx[0]].block
+    full = [x_dev[lay.x_off[i]:lay.x_off[i] + specs[i].numel * 2].view(torch.bfloat16)
+            .view(specs[i].M, specs[i].N) for i in idx]
+    ranges = [shard_rows(specs[i].M, world, bm)[rank] for i in idx]
+    shards = [f[lo:hi] for f, (lo, hi) in zip(full, ranges)]
+    sqg = ShardedQuantGather([(specs[i].M, specs[i].N) for i in idx], (bm, bn), device=dev)
+    # baseline buffers: padded bf16 shards (as FSDP keeps them), the gathered
+    # bf16 weights, and the quantized outputs
+    rows = [-(-(-(-specs[i].M // bm)) // world) * bm for i in idx]
+    pad = [torch.zeros((r, specs[i].N), dtype=torch.bfloat16, device=dev) for r, i in zip(rows, idx)]
+    for p_, sh in zip(pad, shards):
+        p_[:sh.shape[0]].copy_(sh)
+    gathered = [torch.empty((world * r, specs[i].N), dtype=torch.bfloat16, device=dev)
+                for r, i in zip(rows, idx)]
+    outs = [fq._outputs(g[:specs[i].M], (bm, bn)) for g, i in zip(gathered, idx)]
+    base_descs = [fq.make_desc(g[:specs[i].M], y, s_, (bm, bn))
+                  for g, i, (y, s_) in zip(gathered, idx, outs)]
+    base_table = (fq.fp8bq_desc * len(base_descs))(*base_descs)
+    L = fq.lib()
+    stream = torch.cuda.current_stream(dev)
+    sh = ctypes.c_void_p(stream.cuda_stream)
+
+    def step_ours():
+        sqg.run(shards)
+
+    def step_base():
+        for g, p_ in zip(gathered, pad):
+            tdist.all_gather_into_tensor(g, p_)
+        st = L.fp8bq_quantize_batched(base_table, len(base_descs), sh)
+        if st != 0:
+            raise RuntimeError(fq.fp8bq_status_string(st))
+
+    def timed(step):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        dist.barrier()
+        return dist.max(t0.elapsed_time(t1) / 1e3)
+
+    with ClockSampler(dev) as clk:
+        el_ours = timed(step_ours)
+        el_base = timed(step_base)
+    # both ways give the same bytes
+    res = sqg.run(shards)
+    torch.cuda.synchronize()
+    same = all(torch.equal(a.view(torch.uint8), y.view(torch.uint8)) and torch.equal(b, s_)
+               for (a, b), (y, s_) in zip(res, outs))
+    nbytes = sum(specs[i].algorithmic_bytes for i in idx)
+    value = aggregate(nbytes, args.steps, world, el_ours)
+    peak, kind = measured_peak()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "sharded weight sync: quantize shards + all-gather e4m3 codes, GB/s of "
+                      "quantizer bytes of the whole weights",
+            "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": el_ours / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": wl_desc + f"; {len(idx)} weights row-sharded over {world} "
+                                             f"rank(s) in whole block rows", "name": args.workload,
+                       "op": "shard", "bytes_per_step": nbytes,
+                       "gathered_bytes_per_rank_ours": sum(b.codes.numel() + b.descale.numel() * 4
+                                                           for b in sqg.bufs),
+                       "gathered_bytes_per_rank_baseline": sum(g.numel() * 2 for g in gathered)},
+            "baseline_gather_bf16_then_quantize": {
+                "value": aggregate(nbytes, args.steps, world, el_base), "unit": "GB/s",
+                "ms_per_step": el_base / args.steps * 1e3},
+            "same_bytes_both_ways": same,
+            "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
+                         "frac": value / world / peak, "traffic": None, "peak_source": kind},
+            "gpu_launches": None, "clocks": clk.summary()}), flush=True)
+    if world == 1:
+        tdist.destroy_process_group()
+
+
 def run_scale_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc) -> None:
     """Time fp8bq_tensor_scale over every tensor of the workload (one grouped
     call per step): a read-only pass, numel * elem_bytes + 4 bytes per tensor."""
@@ -801,10 +916,12 @@ def main() -> None:
     ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",
                     help="C-ABI calls per step: one grouped call, one per layer, or one per "
                          "tensor")
-    ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale"],
+    ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale", "shard"],
                     default="quantize",
                     help="dequantize: time the reverse map on the quantized workload; "
-                         "tensor_scale: time per-tensor scales of the workload's tensors")
+                         "tensor_scale: time per-tensor scales of the workload's tensors; "
+                         "shard: time quantize-then-gather of row-sharded weights against "
+                         "gather-then-quantize")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="CPU time spent on the oracle baseline (0 = skip)")
     ap.add_argument("--keep-inputs", action="store_true",

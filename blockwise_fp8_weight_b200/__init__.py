@@ -41,6 +41,7 @@ FP8BQ_ERR_DEVICE = 6
 FP8BQ_ERR_DEVICE_TIMEOUT = 7
 FP8BQ_ERR_ALIGN = 8
 FP8BQ_ERR_ARG = 9
+FP8BQ_ERR_DEVICE_UNSAFE = 10
 # fp8bq_path
 FP8BQ_PATH_AUTO = 0
 FP8BQ_PATH_VECTOR = 1
@@ -303,6 +304,21 @@ def make_desc(x, y, s, block=DEFAULT_BLOCK) -> fp8bq_desc:
     return d
 
 
+def _on_stream(stream):
+    """Context in which PyTorch allocates for ``stream``: outputs the library
+    writes on a stream other than the current one are allocated on that
+    stream, so the caching allocator cannot hand their memory to another
+    stream's work while the kernel still writes it."""
+    import contextlib
+
+    import torch
+    if stream is None:
+        return contextlib.nullcontext()
+    if isinstance(stream, int):
+        stream = torch.cuda.ExternalStream(stream)
+    return torch.cuda.stream(stream)
+
+
 def _outputs(x, block):
     import torch
     M, N = x.shape[-2], x.shape[-1]
@@ -322,7 +338,8 @@ def scaled_fp8_blockwise(data_hp, weight_block_size=DEFAULT_BLOCK, stream=None):
     """
     block = tuple(int(b) for b in weight_block_size)
     _check_cuda(data_hp, "data_hp")
-    y, s = _outputs(data_hp, block)
+    with _on_stream(stream):
+        y, s = _outputs(data_hp, block)
     check(fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream),
           "scaled_fp8_blockwise")
     return y, s
@@ -343,7 +360,8 @@ def dequantize_fp8_blockwise(fp8_data, descale, weight_block_size=DEFAULT_BLOCK,
     bm, bn = (int(b) for b in weight_block_size)
     M, N = fp8_data.shape[-2], fp8_data.shape[-1]
     batch = fp8_data.shape[0] if fp8_data.dim() == 3 else 1
-    out = torch.empty(fp8_data.shape, dtype=out_dtype, device=fp8_data.device)
+    with _on_stream(stream):
+        out = torch.empty(fp8_data.shape, dtype=out_dtype, device=fp8_data.device)
     check(fp8bq_dequantize(fp8_data, descale, batch, M, N, bm, bn, out,
                            FP8BQ_BF16 if out_dtype == torch.bfloat16 else FP8BQ_F32, N, M * N,
                            stream), "dequantize_fp8_blockwise")
@@ -359,7 +377,8 @@ def tensor_scales(tensors, stream=None):
     if not tensors:
         raise ValueError("no tensors")
     _check_cuda(tensors[0], "every tensor")
-    out = torch.empty(len(tensors), dtype=torch.float32, device=tensors[0].device)
+    with _on_stream(stream):
+        out = torch.empty(len(tensors), dtype=torch.float32, device=tensors[0].device)
     descs = []
     for t in tensors:
         _check_cuda(t, "every tensor")
@@ -380,7 +399,8 @@ def quant_weights(weights: Iterable, weight_block_size=DEFAULT_BLOCK, stream=Non
     items, descs = [], []
     for name, w in weights:
         _check_cuda(w, name)
-        y, s = _outputs(w, block)
+        with _on_stream(stream):
+            y, s = _outputs(w, block)
         items.append((name, y, s, w))
         descs.append(make_desc(w, y, s, block))
     check(fp8bq_quantize_batched(descs, stream=stream), "quant_weights")

@@ -158,6 +158,23 @@ bool halves_aligned(const fp8bq_desc &D) {
     return true;
 }
 
+// Row class of a tensor on the vector kernel: whole 16-byte vectors; or
+// 8-byte aligned rows loaded into registers; or (FP8BQ_HALVES_RING) the same
+// rows through the shifted cp.async ring (x itself 16-byte aligned, so no
+// copy starts before the tensor, and enough vectors per block row for its
+// extra slots).  Measured on B200 (bf16 4000x4100, 16 such tensors in one
+// call): registers 5270 GB/s, shifted ring 3784 GB/s -- the ring is off.
+#ifndef FP8BQ_HALVES_RING
+#define FP8BQ_HALVES_RING 0
+#endif
+Rows rows_of(const fp8bq_desc &D) {
+    if (vector_aligned(D)) return Rows::Aligned16;
+    const int vec = 16 / esize_of(D.dtype_in);
+    if (FP8BQ_HALVES_RING && (uintptr_t)D.x % 16 == 0 && D.block_n / vec >= kHalvesMinVpr)
+        return Rows::HalvesRing;
+    return Rows::HalvesRegs;
+}
+
 Variant vector_variant(const fp8bq_desc &D) {
     for (Variant v : {Variant::VecT16, Variant::VecT64, Variant::VecTBig})
         if (vector_fits(D, v)) return v;
@@ -365,7 +382,7 @@ void pack_header(DescPack<MAXD> &p) {
 // Launch one group (same variant, dtype and, for vector/TMA, block shape) in
 // chunks that fit the parameter pack and keep the tile count below 2^31.
 template <int MAXD>
-cudaError_t launch_group(Variant v, int es, bool halves, const fp8bq_desc *t,
+cudaError_t launch_group(Variant v, int es, Rows rows, const fp8bq_desc *t,
                          const std::vector<int> &idx, cudaStream_t st) {
     static thread_local DescPack<MAXD> p;  // large: keep it off the stack
     size_t i = 0;
@@ -381,7 +398,7 @@ cudaError_t launch_group(Variant v, int es, bool halves, const fp8bq_desc *t,
             ++i;
         }
         const cudaError_t e = v == Variant::Generic ? launch_generic<MAXD>(es, p, st)
-                                                    : launch_vector<MAXD>(v, es, halves, p, st);
+                                                    : launch_vector<MAXD>(v, es, rows, p, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -421,9 +438,9 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
 struct GroupKey {
     Variant v;
     int es, bm, bn;
-    bool halves;
+    Rows rows;
     bool operator==(const GroupKey &o) const {
-        return v == o.v && es == o.es && bm == o.bm && bn == o.bn && halves == o.halves;
+        return v == o.v && es == o.es && bm == o.bm && bn == o.bn && rows == o.rows;
     }
 };
 
@@ -459,9 +476,10 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         // vector / TMA launches need one block shape; generic ones only one
         // size class (CTA per block for >= 2048 elements, else warp per block)
         const bool big = (int64_t)D.block_m * D.block_n >= 2048;
-        const bool halves = v != Variant::Generic && v != Variant::Tma && !vector_aligned(D);
+        const Rows rows =
+            v != Variant::Generic && v != Variant::Tma ? rows_of(D) : Rows::Aligned16;
         GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? (int)big : D.block_m,
-                   v == Variant::Generic ? 0 : D.block_n, halves};
+                   v == Variant::Generic ? 0 : D.block_n, rows};
         size_t g = 0;
         while (g < keys.size() && !(keys[g] == k)) ++g;
         if (g == keys.size()) {
@@ -479,10 +497,10 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
                     ? launch_tma_group<kMaxDescSmall>(keys[g].es, table, members[g], maps[g], stream)
                     : launch_tma_group<kMaxDescTma>(keys[g].es, table, members[g], maps[g], stream);
         else if (members[g].size() <= (size_t)kMaxDescSmall)
-            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].halves, table,
+            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].rows, table,
                                             members[g], stream);
         else
-            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].halves, table,
+            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].rows, table,
                                             members[g], stream);
         if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
     }
@@ -516,8 +534,11 @@ fp8bq_status check_dequant_desc(const fp8bq_dequant_desc &D, bool *empty) {
 bool dequant_vector_ok(const fp8bq_dequant_desc &D) {
     const int oes = esize_of(D.dtype_out);
     const int64_t obs = D.batch > 1 ? D.out_batch_stride : 0;
+    // the vector kernel numbers its work items (row segments) in 32 bits
+    const uint64_t items = (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll());
     return D.N % 16 == 0 && D.block_n % 16 == 0 && (uintptr_t)D.y_u8 % 16 == 0 &&
-           (uintptr_t)D.out % 16 == 0 && (D.ld_out * oes) % 16 == 0 && (obs * oes) % 16 == 0;
+           (uintptr_t)D.out % 16 == 0 && (D.ld_out * oes) % 16 == 0 && (obs * oes) % 16 == 0 &&
+           items < (1ull << 31);
 }
 
 template <int MAXD>
@@ -531,6 +552,11 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
         p.total = 0;
         while (i < idx.size() && p.n < MAXD) {
             const fp8bq_dequant_desc &D = t[idx[i]];
+            // vector: warp items of 32 x U x 16 codes of a row, numbered in 32 bits
+            const uint64_t items =
+                vector ? (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
+                       : (uint64_t)(D.batch * D.M * D.N);
+            if (vector && p.n > 0 && p.total + items >= (1ull << 32)) break;
             DequantDesc &o = p.d[p.n];
             o.y = D.y_u8;
             o.s = D.descale_f32;
@@ -543,11 +569,10 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.bn = D.block_n;
             o.gm = (int32_t)cdiv(D.M, D.block_m);
             o.gn = (int32_t)cdiv(D.N, D.block_n);
+            o.bm_log2 = is_pow2(D.block_m) ? __builtin_ctz((unsigned)D.block_m) : -1;
+            o.bn_log2 = is_pow2(D.block_n) ? __builtin_ctz((unsigned)D.block_n) : -1;
             o.begin = p.total;
-            // vector: warp items of 32 x 16 codes per row; generic: one element
-            o.items = vector ? (uint64_t)(D.batch * D.M) *
-                                   (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
-                             : (uint64_t)(D.batch * D.M * D.N);
+            o.items = items;
             p.total += o.items;
             ++p.n;
             ++i;
@@ -761,6 +786,9 @@ const char *fp8bq_status_string(fp8bq_status s) {
             return "FP8BQ_ERR_DEVICE_TIMEOUT: a bounded device wait ran out";
         case FP8BQ_ERR_ALIGN: return "FP8BQ_ERR_ALIGN: misaligned input or descale pointer";
         case FP8BQ_ERR_ARG: return "FP8BQ_ERR_ARG: invalid argument";
+        case FP8BQ_ERR_DEVICE_UNSAFE:
+            return "FP8BQ_ERR_DEVICE_UNSAFE: a kernel returned with a tile copy in flight; "
+                   "stop using the GPU";
     }
     return "FP8BQ_?: unknown status";
 }
@@ -776,7 +804,7 @@ fp8bq_status fp8bq_sync_status(cudaStream_t stream) {
         cudaGetLastError();
         return FP8BQ_ERR_DEVICE;
     }
-    return w ? FP8BQ_ERR_DEVICE_TIMEOUT : FP8BQ_OK;
+    return (w & 2u) ? FP8BQ_ERR_DEVICE_UNSAFE : w ? FP8BQ_ERR_DEVICE_TIMEOUT : FP8BQ_OK;
 }
 
 int fp8bq_version(void) { return FP8BQ_VERSION; }

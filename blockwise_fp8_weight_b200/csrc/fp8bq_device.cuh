@@ -19,6 +19,19 @@ __device__ __forceinline__ void pdl_entry() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
+// The two halves of pdl_entry, for kernels that do work touching no global
+// memory the previous kernel may write (shared-memory set-up, prefetching
+// their own kernel-parameter tensor maps) between them.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Bring a TMA tensor map (in kernel-parameter space) into the descriptor
+// cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tensormap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
 
 // ---------------------------------------------------------------- global memory
 
@@ -111,14 +124,43 @@ __device__ __forceinline__ uint32_t quant_f32x4(uint32_t a, uint32_t b, uint32_t
     return o;
 }
 
-// Running max of the magnitudes of two packed bf16 (unsigned halfword max of
-// the sign-cleared bit patterns: for non-negative IEEE values the integer
-// order of the bits is the numeric order).
+// Running maxima of magnitudes.  Two forms, equal for every non-NaN input:
+//   FP8BQ_ABSMAX_FMAX 1: one max.xorsign.abs per pair of bf16 (or per fp32):
+//     the magnitude of the result is max(|m|, |w|) exactly (max does not
+//     round); its sign bit carries no meaning and is cleared when the
+//     maximum is read out (absmax_bits_*).
+//   FP8BQ_ABSMAX_FMAX 0: unsigned integer max of the sign-cleared bit
+//     patterns (for non-negative IEEE values the integer order of the bits is
+//     the numeric order); the running maximum m must have clear sign bits,
+//     as every maximum these functions return has.
+#ifndef FP8BQ_ABSMAX_FMAX
+#define FP8BQ_ABSMAX_FMAX 0
+#endif
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
     uint32_t d;
+#if FP8BQ_ABSMAX_FMAX
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(w));
+#else
     asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(w & 0x7fff7fffu));
+#endif
     return d;
 }
+__device__ __forceinline__ uint32_t absmax_f32(uint32_t m, uint32_t w) {
+#if FP8BQ_ABSMAX_FMAX
+    uint32_t d;
+    asm("max.xorsign.abs.f32 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(w));
+    return d;
+#else
+    return max(m, w & 0x7fffffffu);
+#endif
+}
+// fp32 bit pattern of the larger magnitude of a running bf16x2 maximum, and
+// of a running fp32 maximum.
+__device__ __forceinline__ uint32_t absmax_bits_bf16x2(uint32_t m) {
+    m &= 0x7fff7fffu;
+    return max(m & 0xffffu, m >> 16) << 16;
+}
+__device__ __forceinline__ uint32_t absmax_bits_f32(uint32_t m) { return m & 0x7fffffffu; }
 
 // bf16 halves of a 32-bit word, widened to fp32 (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -149,6 +191,22 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *src, boo
     asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)),
                  "l"(src), "r"(ok ? 16 : 0)
                  : "memory");
+}
+// The same with the number of bytes to read given (0, 8 or 16; the rest of
+// the 16 is zero-filled); src 16-byte aligned.
+__device__ __forceinline__ void cp_async_16_n(void *smem_dst, const void *src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)),
+                 "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+// 8-byte shared-memory load (8-byte aligned address).
+__device__ __forceinline__ uint2 lds_v2(const void *p) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "r"(smem_addr(p))
+                 : "memory");
+    return v;
 }
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");

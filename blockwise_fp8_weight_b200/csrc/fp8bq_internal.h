@@ -5,7 +5,57 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 namespace fp8bq {
+
+// ------------------------------------------------------------------ per-device host state
+//
+// Kernel attributes (the dynamic shared-memory limit), resident CTAs per SM
+// and the SM count are properties of a device: each is computed once per
+// device, with that device current, so one process may drive several GPUs.
+constexpr int kMaxDevices = 64;
+
+inline int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        dev = 0;
+    }
+    return dev;
+}
+
+// A value made once per device (devices beyond kMaxDevices: made on every call).
+template <typename T>
+class PerDevice {
+  public:
+    template <typename F>
+    T get(F &&make) {
+        const int dev = current_device();
+        if (dev < 0 || dev >= kMaxDevices) return make();
+        std::call_once(once_[dev], [&] { val_[dev] = make(); });
+        return val_[dev];
+    }
+
+  private:
+    std::once_flag once_[kMaxDevices];
+    T val_[kMaxDevices];
+};
+
+// Streaming multiprocessors of the current device.
+inline int sm_count() {
+    static PerDevice<int> n;
+    return n.get([] {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, current_device()) !=
+                cudaSuccess ||
+            v <= 0) {
+            cudaGetLastError();
+            v = 148;
+        }
+        return v;
+    });
+}
 
 // The eps floor of the block absmax.  The pages print the floor (absmax =
 // max(max|x|, eps)) but not its value; 1e-10 is this library's reading.
@@ -97,11 +147,21 @@ enum class Variant : int {
     Tma = 4,
 };
 
+// Row alignment classes of the vector kernel (uniform per launch).
+enum class Rows : int {
+    Aligned16 = 0,   // 16-byte aligned rows: cp.async ring of whole vectors
+    HalvesRing = 1,  // 8-byte aligned rows, x 16-byte aligned, >= kHalvesMinVpr vectors
+                     // per block row: cp.async ring of aligned 16-byte copies, shifted rows
+                     // reassembled in shared memory
+    HalvesRegs = 2,  // other 8-byte aligned rows: two 8-byte loads per vector into registers
+};
+// Fewest 16-byte vectors per block row for Rows::HalvesRing (sizes its extra slots).
+constexpr int kHalvesMinVpr = 8;
+
 // Launchers (vector and generic: fp8bq_kernels.cu; TMA: fp8bq_tma.cu).  Each
 // returns cudaSuccess or the launch error.
-// halves: rows only 8-byte aligned (each 16-byte vector moved as two halves)
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
+cudaError_t launch_vector(Variant v, int esize, Rows rows, const DescPack<MAXD> &p,
                           cudaStream_t st);
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);
@@ -111,19 +171,21 @@ template <int MAXD>
 cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st);
 
 // Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
-// grouped launch walks the concatenated work items (a warp-wide row segment
-// of 32 x 16 codes for the vector kernel, one element for the generic one) of
-// all descriptors of a pack.
+// grouped launch walks the concatenated work items (one matrix row for the
+// vector kernel, one element for the generic one) of all descriptors of a
+// pack.
 struct DequantDesc {
     const uint8_t *y;   // [batch, M, N] codes
     const float *s;     // [batch, gm, gn] descales
     void *out;          // matrix b at out + b * obs elements, row stride ldo
     int64_t M, N, ldo, obs;
     int32_t bm, bn, gm, gn;
+    int32_t bm_log2;    // log2(bm) if bm is a power of two, else -1
+    int32_t bn_log2;    // log2(bn) if bn is a power of two, else -1
     uint64_t begin;     // first work item of this descriptor
     uint64_t items;     // work items of this descriptor
 };
-static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
+static_assert(sizeof(DequantDesc) == 96, "DequantDesc layout");
 
 template <int MAXD>
 struct DequantPack {
@@ -136,7 +198,7 @@ static_assert(sizeof(DequantPack<kMaxDescLarge>) < 32000, "kernel parameter limi
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st);
-// 16-byte code chunks per lane per warp work item of the vector dequant kernel
+// 16-byte code chunks per lane in a work item of the vector dequant kernel
 int dequant_unroll();
 
 // Per-tensor scales (fp8bq_scale.cu): the tensors of a pack are cut into

@@ -100,17 +100,27 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // geometry, each 16-byte vector moved as two 8-byte halves; a half beyond
 // the row end reads as zeros (no effect on the absmax) and is not stored.
 //
-// S > 0 (16-byte aligned rows): the loads go through a private ring of S
-// stages per thread in shared memory (cp.async), S - 1 tiles in flight while
-// one is reduced and stored.  S == 0 (HALVES): two register sets, the next
-// tile loaded while the current one is processed (measured faster there than
-// a ring of 8-byte cp.async copies: 4.38-4.65 against 4.10 TB/s).
+// S > 0: the loads go through a ring of S stages in shared memory (cp.async,
+// 16-byte copies), S - 1 tiles in flight while one is reduced and stored;
+// slot i of thread t of stage s is stage[(s * V + i) * CTA + t], so the
+// slots of the vpr lanes of a block row are 16 * vpr contiguous bytes.
+//   16-byte aligned rows: each lane copies its own vector.
+//   HALVES (rows 8-byte aligned, x 16-byte aligned, vpr >= 8): in a row
+//   that starts 8 bytes past a 16-byte boundary ("shifted"), lane cv copies
+//   the aligned 16 bytes that begin 8 bytes before its vector (the tail of
+//   its left neighbour's vector, then its own first half), and its vector is
+//   read back from shared memory 8 bytes into its slot: its first half, then
+//   the head of lane cv + 1's slot; the last lane of the row copies that
+//   second half into a per-row extra slot.  Every copy starts on a 16-byte
+//   boundary; bytes beyond the row end are zero-filled, not read.
+// S == 0 (HALVES, other cases): two register sets, the next tile loaded
+// straight into registers (two 8-byte loads per vector) while the current one
+// is processed.
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, int S>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     dev::pdl_entry();
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
-    static_assert(!(HALVES && S > 0), "the cp.async ring takes 16-byte vectors only");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -129,15 +139,36 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     const int colv = cv * VEC;
     const uint32_t shfl_mask =
         TEAM >= 32 ? 0xffffffffu : (((1u << TEAM) - 1u) << ((threadIdx.x & 31) & ~(TEAM - 1)));
-    int d = 0;  // current descriptor; advances monotonically with the tile id
+    TileCursor<ESIZE, G, MAXD> walk(p, stride);  // the tiles this team loads, in order
 
     // upper 8-byte half of this lane's vector inside the row (HALVES only)
     auto hi_ok = [&](const Tile &T) { return colv + VEC / 2 < T.cols; };
-    auto store = [&](const uint4 &v, uint64_t rr, uint8_t *dst, const Tile &T) {
+    auto store = [&](const uint4 &v, uint64_t rr, uint8_t *dst, bool hi) {
         if constexpr (HALVES)
-            vec_quant_store_halves<ESIZE>(v, rr, dst, hi_ok(T));
+            vec_quant_store_halves<ESIZE>(v, rr, dst, hi);
         else
             vec_quant_store<ESIZE>(v, rr, dst);
+    };
+    // Every slot of every lane of the team lies inside the tile (the same for
+    // the whole team): the interior tiles skip the per-vector bounds checks.
+    auto is_full = [&](const Tile &T) { return T.rows >= V * rstep && T.cols >= vpr * VEC; };
+    // Quantize and store slot i of every lane for i < NB (the slots of blocks
+    // inside the matrix), with the reciprocal rr(i).
+    auto store_all = [&](const uint4 (&R)[V], const Tile &T, int nb, auto rr_of) {
+        uint8_t *dst = T.dst + (int64_t)row0 * T.ldy + colv;
+        const int64_t ystep = (int64_t)rstep * T.ldy;
+        if (is_full(T)) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) store(R[i], rr_of(i), dst + i * ystep, true);
+        } else {
+            const bool hi = hi_ok(T);
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                if (i >= nb) break;
+                if (row0 + i * rstep < T.rows && colv < T.cols)
+                    store(R[i], rr_of(i), dst + i * ystep, hi);
+            }
+        }
     };
 
     auto load = [&](uint4 (&R)[V], const Tile &T) {
@@ -177,13 +208,8 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         float r[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + 2 * i);
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            if (i * bm >= T.rows) break;  // blocks below the matrix
-            const int rr = row0 + i * rstep;
-            if (rr < T.rows && colv < T.cols)
-                store(R[i], dev::splat2(r[i]), T.dst + (int64_t)rr * T.ldy + colv, T);
-        }
+        // slots of blocks below the matrix are neither quantized nor stored
+        store_all(R, T, (T.rows + bm - 1) / bm, [&](int i) { return dev::splat2(r[i]); });
         const int slot = lane >> 1;
         if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
       }
@@ -209,34 +235,91 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         float s, r;
         dev::block_scale(m, kEps, s, r);
         const uint64_t r2 = dev::splat2(r);
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int rr = row0 + i * rstep;
-            if (rr < T.rows && colv < T.cols)
-                store(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv, T);
-        }
+        store_all(R, T, V, [&](int) { return r2; });
         if (lane == 0) *T.sdst = s;
     };
 
     if constexpr (S > 0) {
         extern __shared__ __align__(1024) uint8_t ring[];  // dynamic shared memory
         uint4 *const stage = reinterpret_cast<uint4 *>(ring);  // [S][V][CTA] 16-byte vectors
+        // HALVES: [S][V][CTA / kHalvesMinVpr] extra slots, one per row of a row step
+        uint4 *const extra = stage + S * V * CTA;
+        constexpr int XR = CTA / kHalvesMinVpr;
+        const bool last_lane = cv == vpr - 1;
+        const int xrow = threadIdx.x / vpr;  // this thread's row within the CTA's row step
+        // an aligned source for copies that read nothing (x is 16-byte aligned)
+        auto safe = [](const Tile &T) {
+            return (const char *)((uintptr_t)T.src & ~(uintptr_t)15);
+        };
         auto issue = [&](int s, const Tile &T) {
+            const bool full = is_full(T);
+            const char *src0 = T.src + ((int64_t)row0 * T.ld + colv) * ESIZE;
+            const int64_t xstep = (int64_t)rstep * T.ld * ESIZE;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int r = row0 + i * rstep;
-                const bool ok = r < T.rows && colv < T.cols;
-                const char *src = ok ? T.src + ((int64_t)r * T.ld + colv) * ESIZE : T.src;
-                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], src, ok);
+                uint4 *slot = &stage[(s * V + i) * CTA + threadIdx.x];
+                if constexpr (HALVES) {
+                    const bool rok = r < T.rows;
+                    const uintptr_t row = (uintptr_t)T.src + (uintptr_t)((int64_t)r * T.ld * ESIZE);
+                    const uintptr_t a = row + (uintptr_t)(colv * ESIZE);
+                    const bool shifted = (row & 8) != 0;
+                    const bool lo = rok && colv < T.cols;           // first half in the row
+                    const bool hi = rok && colv + VEC / 2 < T.cols;  // second half in the row
+                    const char *al = (const char *)(a & ~(uintptr_t)15);
+                    if (shifted) {
+                        // [a - 8, a + 8): the left lane's second half, then ours; only
+                        // the left lane's part when ours lies beyond the row end
+                        const bool left = rok && colv - VEC / 2 < T.cols;
+                        const int n = lo ? 16 : left ? 8 : 0;
+                        dev::cp_async_16_n(slot, n ? al : safe(T), n);
+                        if (last_lane)  // our second half, [a + 8, a + 16)
+                            dev::cp_async_16_n(&extra[(s * V + i) * XR + xrow],
+                                               hi ? al + 16 : safe(T), hi ? 8 : 0);
+                    } else {
+                        const int n = hi ? 16 : lo ? 8 : 0;
+                        dev::cp_async_16_n(slot, n ? al : safe(T), n);
+                    }
+                } else {
+                    const bool ok = full || (r < T.rows && colv < T.cols);
+                    dev::cp_async_16(slot, ok ? src0 + i * xstep : T.src, ok);
+                }
             }
             dev::cp_async_commit();
+        };
+        // Read this thread's vectors of stage s (HALVES: after every lane's
+        // copies have landed, reassembled across the slots of a shifted row).
+        auto fetch = [&](int s, const Tile &T, uint4 (&R)[V]) {
+            if constexpr (HALVES) {
+                // the copies of the row's other lanes (same team, same warp) are visible
+                __syncwarp(shfl_mask);
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int r = row0 + i * rstep;
+                    const uint4 *slot = &stage[(s * V + i) * CTA + threadIdx.x];
+                    const bool shifted =
+                        (((uintptr_t)T.src + (uintptr_t)((int64_t)r * T.ld * ESIZE)) & 8) != 0;
+                    if (shifted) {
+                        const uint2 lo = dev::lds_v2(reinterpret_cast<const char *>(slot) + 8);
+                        const uint2 up = dev::lds_v2(last_lane ? (const void *)&extra[(s * V + i) * XR + xrow]
+                                                               : (const void *)(slot + 1));
+                        R[i] = make_uint4(lo.x, lo.y, up.x, up.y);
+                    } else {
+                        R[i] = *slot;
+                    }
+                }
+                __syncwarp(shfl_mask);  // every lane has read the stage before any refills it
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
+            }
         };
         Tile Ts[S];
         uint32_t tn = t;  // next tile to issue; t: next tile to process
 #pragma unroll
         for (int s = 0; s < S; ++s) {
             if (tn < p.total_tiles) {
-                Ts[s] = make_tile<ESIZE, G>(p, tn, d);
+                Ts[s] = walk.next(tn);
                 issue(s, Ts[s]);
             } else {
                 dev::cp_async_commit();  // empty group: keeps the wait count uniform
@@ -254,11 +337,10 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
                 }
                 dev::cp_async_wait<S - 1>();  // this thread's copies of stage s have landed
                 uint4 R[V];
-#pragma unroll
-                for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
+                fetch(s, Ts[s], R);
                 process(R, Ts[s], it++);  // consumes R: the stage is free again
                 if (tn < p.total_tiles) {
-                    Ts[s] = make_tile<ESIZE, G>(p, tn, d);
+                    Ts[s] = walk.next(tn);
                     issue(s, Ts[s]);
                 } else {
                     dev::cp_async_commit();
@@ -272,7 +354,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     }
 
     uint4 A[V], B[V];
-    Tile ta = make_tile<ESIZE, G>(p, t, d);
+    Tile ta = walk.next(t);
     load(A, ta);
     uint32_t it = 0;
     while (true) {
@@ -280,7 +362,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         const bool h1 = t1 < p.total_tiles;
         Tile tb;
         if (h1) {
-            tb = make_tile<ESIZE, G>(p, t1, d);
+            tb = walk.next(t1);
             load(B, tb);
         }
         process(A, ta, it++);
@@ -288,7 +370,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         const uint32_t t2 = t1 + stride;
         const bool h2 = t2 < p.total_tiles;
         if (h2) {
-            ta = make_tile<ESIZE, G>(p, t2, d);
+            ta = walk.next(t2);
             load(A, ta);
         }
         process(B, tb, it++);
@@ -392,44 +474,48 @@ __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ Des
 
 namespace {
 
-template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
+// RING: the cp.async ring (16-byte aligned rows, or HALVES rows that the
+// shifted ring can take); else the register path (HALVES only).
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, bool RING>
 cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
-    constexpr int S = HALVES ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
-    constexpr size_t smem = (size_t)S * V * CTA * 16;
+    static_assert(RING || HALVES, "16-byte aligned rows always take the ring");
+    constexpr int S = !RING ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
+    constexpr size_t smem =
+        (size_t)S * V * CTA * 16 + (HALVES ? (size_t)S * V * (CTA / kHalvesMinVpr) * 16 : 0);
     auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES, S>;
-    if constexpr (smem > 48 * 1024) {
-        static cudaError_t attr =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (attr != cudaSuccess) return attr;
-    }
-    static int occ = resident_ctas(kern, CTA, smem);
-    const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, occ);
+    static PerDevice<KernelSetup> setup;
+    const KernelSetup ks = setup.get([&] { return setup_kernel(kern, CTA, smem); });
+    if (ks.attr != cudaSuccess) return ks.attr;
+    const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, ks.occ);
     return launch_kernel(kern, grid, CTA, smem, st, p);
 }
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
-cudaError_t launch_vector_t(bool halves, const DescPack<MAXD> &p, cudaStream_t st) {
-    return halves ? launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true>(p, st)
-                  : launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, false>(p, st);
+cudaError_t launch_vector_t(Rows rows, const DescPack<MAXD> &p, cudaStream_t st) {
+    switch (rows) {
+        case Rows::Aligned16: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, false, true>(p, st);
+        case Rows::HalvesRing: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true, true>(p, st);
+        default: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true, false>(p, st);
+    }
 }
 
 }  // namespace
 
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
+cudaError_t launch_vector(Variant v, int esize, Rows rows, const DescPack<MAXD> &p,
                           cudaStream_t st) {
     if (esize == 2) {
         switch (v) {
-            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(halves, p, st);
-            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(halves, p, st);
-            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(halves, p, st);
+            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(rows, p, st);
+            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(rows, p, st);
+            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(rows, p, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (v) {
-        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(halves, p, st);
-        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(halves, p, st);
-        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(halves, p, st);
+        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(rows, p, st);
+        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(rows, p, st);
+        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(rows, p, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -439,33 +525,25 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
     // blocks of >= 2048 elements take one CTA each (the host groups generic
     // tensors by this size class, so it is uniform per launch)
     const bool cta = (int64_t)p.d[0].bm * p.d[0].bn >= 2048;
+    // one occupancy record per kernel (the four kernels share a type, so a
+    // static inside a shared helper would be shared too)
+    static PerDevice<int> occ_cta2, occ_warp2, occ_cta4, occ_warp4;
+    auto go = [&](auto kern, PerDevice<int> &occ, int tiles_per_cta) {
+        const int o = occ.get([&] { return resident_ctas(kern, 256, 0); });
+        return launch_kernel(kern, grid_for(p.total_tiles, tiles_per_cta, o), 256, 0, st, p);
+    };
     cudaError_t e;
-    if (esize == 2) {
-        if (cta) {
-            static int occ = resident_ctas(k_generic_cta<2, MAXD>, 256, 0);
-            e = launch_kernel(k_generic_cta<2, MAXD>, grid_for(p.total_tiles, 1, occ), 256, 0, st,
-                              p);
-        } else {
-            static int occ = resident_ctas(k_generic<2, MAXD>, 256, 0);
-            e = launch_kernel(k_generic<2, MAXD>, grid_for(p.total_tiles, 8, occ), 256, 0, st, p);
-        }
-    } else {
-        if (cta) {
-            static int occ = resident_ctas(k_generic_cta<4, MAXD>, 256, 0);
-            e = launch_kernel(k_generic_cta<4, MAXD>, grid_for(p.total_tiles, 1, occ), 256, 0, st,
-                              p);
-        } else {
-            static int occ = resident_ctas(k_generic<4, MAXD>, 256, 0);
-            e = launch_kernel(k_generic<4, MAXD>, grid_for(p.total_tiles, 8, occ), 256, 0, st, p);
-        }
-    }
+    if (esize == 2)
+        e = cta ? go(k_generic_cta<2, MAXD>, occ_cta2, 1) : go(k_generic<2, MAXD>, occ_warp2, 8);
+    else
+        e = cta ? go(k_generic_cta<4, MAXD>, occ_cta4, 1) : go(k_generic<4, MAXD>, occ_warp4, 8);
     return e;
 }
 
-template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, bool,
+template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, Rows,
                                                   const DescPack<kMaxDescSmall> &,
                                                   cudaStream_t);
-template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, bool,
+template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, Rows,
                                                   const DescPack<kMaxDescLarge> &,
                                                   cudaStream_t);
 template cudaError_t launch_generic<kMaxDescSmall>(int, const DescPack<kMaxDescSmall> &,

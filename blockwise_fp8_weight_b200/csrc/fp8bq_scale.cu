@@ -69,13 +69,13 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
 #pragma unroll
             for (int j = 0; j < LOADS; ++j) {
                 if constexpr (ESIZE == 2) {
-                    const uint32_t a = dev::absmax_bf16x2(dev::absmax_bf16x2(0u, v[j].x), v[j].y);
-                    const uint32_t b = dev::absmax_bf16x2(dev::absmax_bf16x2(0u, v[j].z), v[j].w);
-                    const uint32_t c = dev::absmax_bf16x2(a, b);
-                    m = max(m, max(c & 0xffffu, c >> 16) << 16);
+                    const uint32_t a = dev::absmax_bf16x2(v[j].x & 0x7fff7fffu, v[j].y);
+                    const uint32_t b = dev::absmax_bf16x2(v[j].z & 0x7fff7fffu, v[j].w);
+                    m = max(m, dev::absmax_bits_bf16x2(dev::absmax_bf16x2(a, b)));
                 } else {
-                    m = max(m, max(v[j].x & 0x7fffffffu, v[j].y & 0x7fffffffu));
-                    m = max(m, max(v[j].z & 0x7fffffffu, v[j].w & 0x7fffffffu));
+                    const uint32_t a = dev::absmax_f32(v[j].x & 0x7fffffffu, v[j].y);
+                    const uint32_t b = dev::absmax_f32(v[j].z & 0x7fffffffu, v[j].w);
+                    m = max(m, dev::absmax_bits_f32(dev::absmax_f32(a, b)));
                 }
             }
         } else {
@@ -106,14 +106,7 @@ __global__ void k_scale_finalize(float *scale_out, int n) {
 
 template <int MAXD>
 cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t st) {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
-    }
-    const uint64_t cap = (uint64_t)sms * 8;
+    const uint64_t cap = (uint64_t)sm_count() * 8;
     const unsigned grid = (unsigned)(p.total < cap ? (p.total ? p.total : 1) : cap);
     return esize == 2 ? launch_kernel(k_scale_amax<2, MAXD>, grid, 256, 0, st, p)
                       : launch_kernel(k_scale_amax<4, MAXD>, grid, 256, 0, st, p);

@@ -21,26 +21,12 @@ struct Tile {
     int gn;           // descale row length (blocks per matrix row)
 };
 
-// Tile t of a launch.  A tile is G vertically adjacent blocks of one matrix
-// (G = 1 except for the small-block vector kernel); rows counts the valid
-// rows of all G blocks and sdst points at the first block's descale.
-template <int ESIZE, int G = 1, int MAXD, int H = 1>
-__device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d,
-                                          int g_rt = 1) {
-    while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
-    const TileDesc &D = p.d[d];
-    const uint32_t local = t - D.tile_begin;
-    // G is the compile-time group; g_rt a run-time one (used when G == 0);
-    // H blocks side by side along N (the paired TMA kernel)
-    const uint32_t grp = G == 0 ? (uint32_t)g_rt : (uint32_t)G;
-    const uint32_t gmu = grp == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + grp - 1) / grp;
-    const uint32_t gnu = H == 1 ? (uint32_t)D.gn : ((uint32_t)D.gn + H - 1) / H;
-    const uint32_t per = gmu * gnu;
-    const uint32_t b = local / per;
-    const uint32_t rem = local - b * per;
-    const uint32_t bgi = rem / gnu;
-    const uint32_t bi = bgi * grp;
-    const uint32_t bj = (rem - bgi * gnu) * H;
+// The tile whose first block is (bi, bj) of matrix b of descriptor D: grp
+// vertically stacked blocks (H side by side); rows / cols count the valid
+// extent of all of them and sdst points at the first block's descale.
+template <int ESIZE, int H = 1>
+__device__ __forceinline__ Tile tile_at(const TileDesc &D, uint32_t b, uint32_t bi, uint32_t bj,
+                                        uint32_t grp) {
     const int64_t r0 = (int64_t)bi * D.bm, c0 = (int64_t)bj * D.bn;
     Tile T;
     T.src = (const char *)D.x + ((int64_t)b * D.xbs + r0 * D.ld + c0) * ESIZE;
@@ -57,6 +43,85 @@ __device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, i
     return T;
 }
 
+// Tile t of a launch.  A tile is G vertically adjacent blocks of one matrix
+// (G = 1 except for the small-block kernels); d is a cursor into the
+// descriptor table that only moves forward (tile ids grow along every walk).
+template <int ESIZE, int G = 1, int MAXD, int H = 1>
+__device__ __forceinline__ Tile make_tile(const DescPack<MAXD> &p, uint32_t t, int &d,
+                                          int g_rt = 1) {
+    while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
+    const TileDesc &D = p.d[d];
+    const uint32_t local = t - D.tile_begin;
+    // G is the compile-time group; g_rt a run-time one (used when G == 0);
+    // H blocks side by side along N (the paired TMA kernel)
+    const uint32_t grp = G == 0 ? (uint32_t)g_rt : (uint32_t)G;
+    const uint32_t gmu = grp == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + grp - 1) / grp;
+    const uint32_t gnu = H == 1 ? (uint32_t)D.gn : ((uint32_t)D.gn + H - 1) / H;
+    const uint32_t per = gmu * gnu;
+    const uint32_t b = local / per;
+    const uint32_t rem = local - b * per;
+    const uint32_t bgi = rem / gnu;
+    return tile_at<ESIZE, H>(D, b, bgi * grp, (rem - bgi * gnu) * H, grp);
+}
+
+// The tiles t0, t0 + stride, t0 + 2 stride, ... of one team, visited in
+// order.  make_tile pays two integer divisions per tile; here the position
+// (matrix b, block-group row, block column) advances by the stride written in
+// the mixed radix of the current descriptor (two compares, a few adds), and
+// divisions are paid only when the walk enters another descriptor.
+template <int ESIZE, int G, int MAXD>
+struct TileCursor {
+    const DescPack<MAXD> &p;
+    const uint32_t stride;
+    int d = 0;
+    bool started = false;
+    uint32_t local = 0, b = 0, bgi = 0, bj = 0;  // position within descriptor d
+    uint32_t gmu = 1, gnu = 1;                     // its block-group rows and block columns
+    uint32_t sa = 0, sb = 0, sc = 0;               // the stride in that radix
+
+    __device__ __forceinline__ TileCursor(const DescPack<MAXD> &pk, uint32_t s) : p(pk), stride(s) {}
+
+    __device__ __forceinline__ void seek(uint32_t t) {
+        while (t >= p.d[d].tile_begin + p.d[d].tiles) ++d;
+        const TileDesc &D = p.d[d];
+        gmu = G == 1 ? (uint32_t)D.gm : ((uint32_t)D.gm + G - 1) / G;
+        gnu = (uint32_t)D.gn;
+        const uint32_t per = gmu * gnu;
+        local = t - D.tile_begin;
+        b = local / per;
+        uint32_t rem = local - b * per;
+        bgi = rem / gnu;
+        bj = rem - bgi * gnu;
+        sa = stride / per;
+        rem = stride - sa * per;
+        sb = rem / gnu;
+        sc = rem - sb * gnu;
+    }
+
+    // The tile t (< total): the first call seeks, later ones must pass the
+    // previous t + stride.
+    __device__ __forceinline__ Tile next(uint32_t t) {
+        if (!started) {
+            started = true;
+            seek(t);
+        } else {
+            local += stride;
+            if (local >= p.d[d].tiles) {
+                seek(t);
+            } else {
+                bj += sc;
+                uint32_t c = bj >= gnu ? 1u : 0u;
+                bj -= c * gnu;
+                bgi += sb + c;
+                c = bgi >= gmu ? 1u : 0u;
+                bgi -= c * gmu;
+                b += sa + c;
+            }
+        }
+        return tile_at<ESIZE>(p.d[d], b, bgi * G, bj, G);
+    }
+};
+
 // absmax bits of V 16-byte vectors: four independent running maxima (one per
 // 32-bit lane of the vectors) so the max chains overlap, merged at the end.
 template <int ESIZE, int V>
@@ -70,25 +135,25 @@ __device__ __forceinline__ uint32_t tile_absmax(const uint4 (&R)[V]) {
             m2 = dev::absmax_bf16x2(m2, R[i].z);
             m3 = dev::absmax_bf16x2(m3, R[i].w);
         } else {
-            m0 = max(m0, R[i].x & 0x7fffffffu);
-            m1 = max(m1, R[i].y & 0x7fffffffu);
-            m2 = max(m2, R[i].z & 0x7fffffffu);
-            m3 = max(m3, R[i].w & 0x7fffffffu);
+            m0 = dev::absmax_f32(m0, R[i].x);
+            m1 = dev::absmax_f32(m1, R[i].y);
+            m2 = dev::absmax_f32(m2, R[i].z);
+            m3 = dev::absmax_f32(m3, R[i].w);
         }
     }
     if constexpr (ESIZE == 2)
         return dev::absmax_bf16x2(dev::absmax_bf16x2(m0, m1), dev::absmax_bf16x2(m2, m3));
     else
-        return max(max(m0, m1), max(m2, m3));
+        return dev::absmax_f32(dev::absmax_f32(m0, m1), dev::absmax_f32(m2, m3));
 }
 
-// fp32 bit pattern of the absmax accumulated by vec_absmax / tile_absmax
+// fp32 bit pattern of the absmax accumulated by tile_absmax
 template <int ESIZE>
 __device__ __forceinline__ uint32_t absmax_to_f32_bits(uint32_t m) {
     if constexpr (ESIZE == 2)
-        return max(m & 0xffffu, m >> 16) << 16;
+        return dev::absmax_bits_bf16x2(m);
     else
-        return m;
+        return dev::absmax_bits_f32(m);
 }
 
 // Scales of V blocks whose absmax bits m[0..V-1] every lane of an aligned
@@ -128,17 +193,6 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
 
 // ------------------------------------------------------------------ grid sizing (host)
 
-inline int sm_count() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <typename K>
 inline int resident_ctas(K kernel, int threads, size_t smem) {
     int n = 0;
@@ -146,6 +200,22 @@ inline int resident_ctas(K kernel, int threads, size_t smem) {
         n < 1)
         n = 1;
     return n;
+}
+
+// Set-up of one kernel on one device: the dynamic shared-memory limit (when
+// above the 48 KB default) and the resident CTAs per SM it allows.
+struct KernelSetup {
+    cudaError_t attr;
+    int occ;
+};
+
+template <typename K>
+inline KernelSetup setup_kernel(K kernel, int threads, size_t smem) {
+    KernelSetup s{cudaSuccess, 1};
+    if (smem > 48 * 1024)
+        s.attr = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (s.attr == cudaSuccess) s.occ = resident_ctas(kernel, threads, smem);
+    return s;
 }
 
 inline unsigned grid_for(uint32_t work_units, int units_per_cta, int ctas_per_sm) {

@@ -8,8 +8,10 @@
 
 namespace fp8bq {
 
-// Bit 0: a consumer or producer wait ran out.  Bit 1: the end-of-kernel drain
-// of in-flight TMA copies ran out.
+// Bit 0: a consumer or producer wait ran out (that launch's outputs are
+// incomplete).  Bit 1: the end-of-kernel drain of in-flight TMA copies ran
+// out, so a copy may land in shared memory after the CTA has exited
+// (reported as FP8BQ_ERR_DEVICE_UNSAFE: nothing run since can be trusted).
 __device__ uint32_t g_error_word;
 
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
@@ -60,7 +62,7 @@ enum { MODE_ONE = 0, MODE_SUB = 1, MODE_CTA = 2 };
 template <int ESIZE, int STAGES, int MODE, int MAXD, bool EF>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_SM)
     k_tma(const __grid_constant__ TmaPack<MAXD> P) {
-    dev::pdl_entry();
+    dev::pdl_launch_dependents();
     constexpr int VEC = 16 / ESIZE;
     constexpr int STAGE_BYTES = 128 * 128 * ESIZE;
     constexpr int V = STAGE_BYTES / 16 / kTmaConsumerThreads;
@@ -89,7 +91,13 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         }
         abort_flag = 0;
         dev::fence_mbar_init();
+        // the map of this CTA's first tile, fetched while the previous kernel
+        // of the stream may still be running (the maps are kernel parameters)
+        int d0 = 0;
+        while (d0 + 1 < p.n && blockIdx.x >= p.d[d0].tile_begin + p.d[d0].tiles) ++d0;
+        dev::prefetch_tensormap(&P.maps[d0]);
     }
+    dev::pdl_wait();  // the previous kernel has completed; its writes are visible
     __syncthreads();
 
     const int bm = p.d[0].bm, bn = p.d[0].bn, grp = p.group;
@@ -285,7 +293,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
 template <int STAGES, int MAXD, bool EF>
 __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
     k_tma_pair(const __grid_constant__ TmaPack<MAXD> P) {
-    dev::pdl_entry();
+    dev::pdl_launch_dependents();
     constexpr int ESIZE = 2, VEC = 8, BN = 128, BM = 128;
     constexpr int COLS = 2 * BN;                           // tile columns
     constexpr int STAGE_BYTES = BM * COLS * ESIZE;         // 64 KB
@@ -315,7 +323,13 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
         }
         abort_flag = 0;
         dev::fence_mbar_init();
+        // the map of this CTA's first tile, fetched while the previous kernel
+        // of the stream may still be running (the maps are kernel parameters)
+        int d0 = 0;
+        while (d0 + 1 < p.n && blockIdx.x >= p.d[d0].tile_begin + p.d[d0].tiles) ++d0;
+        dev::prefetch_tensormap(&P.maps[d0]);
     }
+    dev::pdl_wait();  // the previous kernel has completed; its writes are visible
     __syncthreads();
 
     if (warp == 0) {
@@ -417,12 +431,12 @@ template <int ESIZE, int STAGES, int MODE, int MAXD, bool EF>
 cudaError_t launch_tma_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     constexpr size_t smem = (size_t)STAGES * 128 * 128 * ESIZE;
     auto kern = k_tma<ESIZE, STAGES, MODE, MAXD, EF>;
-    static cudaError_t attr =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (attr != cudaSuccess) return attr;
-    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
-                         st, p);
+    static PerDevice<KernelSetup> setup;
+    const KernelSetup ks =
+        setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
+    if (ks.attr != cudaSuccess) return ks.attr;
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ), 32 + kTmaConsumerThreads,
+                         smem, st, p);
 }
 
 // The L2 policy of the tile loads is a template parameter, so the default
@@ -438,12 +452,12 @@ cudaError_t launch_tma_pair_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     constexpr int S = FP8BQ_TMA_PAIR_STAGES;
     constexpr size_t smem = (size_t)S * 128 * 256 * 2;
     auto kern = k_tma_pair<S, MAXD, EF>;
-    static cudaError_t attr =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (attr != cudaSuccess) return attr;
-    static int occ = resident_ctas(kern, 32 + kTmaConsumerThreads, smem);
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, occ), 32 + kTmaConsumerThreads, smem,
-                         st, p);
+    static PerDevice<KernelSetup> setup;
+    const KernelSetup ks =
+        setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
+    if (ks.attr != cudaSuccess) return ks.attr;
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ), 32 + kTmaConsumerThreads,
+                         smem, st, p);
 }
 }  // namespace
 

@@ -9,10 +9,15 @@ of the 2 bytes per element of bf16.  Blocks are independent, so quantizing row
 shards whose boundaries fall on block rows yields exactly the bytes of
 quantizing the whole matrix.
 
-Shards are whole block rows (``shard_rows``): rank r holds rows
-[r * R, min((r + 1) * R, M)) of the [M, N] weight, R a multiple of block_m.
-A shard boundary inside a block row would need the boundary rows exchanged
-before quantizing; such shardings are refused.
+Shards of whole block rows (``shard_rows``): rank r holds rows
+[r * R, min((r + 1) * R, M)) of the [M, N] weight, R a multiple of block_m;
+each rank quantizes its own rows.  Shards of any row ranges (``row_chunks``,
+e.g. an even split of M over the ranks, whose boundaries may fall inside a
+block row): a block row belongs to the rank holding its first row, and the
+rows of it held by later ranks travel to that rank first (a halo exchange of
+fewer than block_m rows per rank, ``exchange_halo``); each rank then
+quantizes its block rows and the ranks broadcast their codes into every
+rank's output (``quantize_and_allgather_rows``).
 
 Data movement: the gather output is one buffer of ``world`` equal slots of R
 rows (``GatherBuffers``); rank r's slot is where its shard's codes go, so the
@@ -177,3 +182,207 @@ def quantize_and_allgather(shard, M: int, weight_block_size: Sequence[int] = (12
         _gather_in_place(buf, rank, group)
         y, s = buf.whole()
         return y.view(torch.float8_e4m3fn), s
+
+
+class ShardedQuantGather:
+    """``quant_weights`` over row-sharded weights, with buffers kept between
+    calls (a trainer syncs the same parameters every step).
+
+    For weights of shapes ``[(M, N), ...]``: ``run(shards)`` quantizes every
+    rank's shard of every weight in ONE grouped launch of the library, each
+    straight into its slot of that weight's gather buffer, then all-gathers
+    each weight's codes and descales in place.  Returns ``[(fp8_data [M, N],
+    descale [gm, gn]), ...]`` views of the buffers (valid until the next
+    ``run``)."""
+
+    def __init__(self, shapes: Sequence[tuple[int, int]],
+                 weight_block_size: Sequence[int] = (128, 128), group=None, device=None):
+        import torch
+        import torch.distributed as dist
+        self.block = tuple(int(b) for b in weight_block_size)
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+        self.shapes = [(int(M), int(N)) for M, N in shapes]
+        self.ranges = [shard_rows(M, self.world, self.block[0])[self.rank]
+                       for M, _ in self.shapes]
+        self.bufs = [gather_buffers(M, N, self.block, self.world, dev) for M, N in self.shapes]
+
+    def run(self, shards, stream=None):
+        import contextlib
+
+        import torch
+
+        from . import check, fp8bq_quantize_batched, make_desc
+        if len(shards) != len(self.shapes):
+            raise ValueError(f"{len(shards)} shards for {len(self.shapes)} weights")
+        ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+        with ctx:
+            descs = []
+            for x, (M, N), (lo, hi), buf in zip(shards, self.shapes, self.ranges, self.bufs):
+                _check_shard("the shard is", self.rank, x.shape, (hi - lo, N))
+                if hi > lo and N > 0:
+                    yc, sc = buf.slot(self.rank, lo, hi)
+                    descs.append(make_desc(x, yc, sc, self.block))
+            if descs:
+                check(fp8bq_quantize_batched(descs), "ShardedQuantGather")
+            out = []
+            for (M, N), buf in zip(self.shapes, self.bufs):
+                if M > 0 and N > 0:
+                    _gather_in_place(buf, self.rank, self.group)
+                y, s = buf.whole()
+                out.append((y.view(torch.float8_e4m3fn), s))
+            return out
+
+
+# ---------------------------------------------------------------- any row split
+
+
+def row_chunks(M: int, world: int) -> list[tuple[int, int]]:
+    """Row range [lo, hi) of every rank for an even split of M rows
+    (ceil(M / world) rows per rank, the last ranks fewer or none), as a
+    dim-0 sharding of a parameter does: boundaries need not fall on block
+    rows."""
+    if M < 0 or world < 1:
+        raise ValueError("need M >= 0, world >= 1")
+    per = -(-M // world)
+    return [(min(r * per, M), min((r + 1) * per, M)) for r in range(world)]
+
+
+def owned_block_rows(ranges, rank: int, block_m: int) -> tuple[int, int]:
+    """Block rows [kb, ke) whose first row lies in ``rank``'s range: the
+    block rows that rank quantizes."""
+    lo, hi = ranges[rank]
+    if hi <= lo:
+        return (0, 0)
+    return (-(-lo // block_m), -(-hi // block_m))
+
+
+def _check_ranges(ranges, M: int, world: int) -> None:
+    if len(ranges) != world:
+        raise ValueError(f"{len(ranges)} row ranges for {world} ranks")
+    at = 0
+    for lo, hi in ranges:
+        if lo != at or hi < lo:
+            raise ValueError(f"row ranges must tile [0, M) in rank order: {ranges}")
+        at = hi
+    if at != M:
+        raise ValueError(f"row ranges end at {at}, not at M = {M}")
+
+
+def exchange_halo(shard, ranges, M: int, block_m: int, group=None):
+    """Gather the rows this rank's block rows need from the ranks after it.
+
+    ``shard``: this rank's rows [lo, hi) of the [M, N] weight (any device the
+    process group serves).  Every rank sends its head -- its rows before its
+    first block-row boundary, fewer than block_m, which belong to a block
+    row that starts on an earlier rank -- in one all-gather of
+    [world, block_m - 1, N] rows.  Returns ``(rows, kb, ke)``: the rows
+    [kb * block_m, min(ke * block_m, M)) of the weight (a view of ``shard``
+    when the shard already holds exactly them, else one new tensor) and this
+    rank's block rows [kb, ke)."""
+    import torch
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    _check_ranges(ranges, M, world)
+    lo, hi = ranges[rank]
+    N = int(shard.shape[-1])
+    if tuple(shard.shape) != (hi - lo, N):
+        raise ValueError(f"rank {rank}: the shard is {tuple(shard.shape)}, expected {(hi - lo, N)}")
+    kb, ke = owned_block_rows(ranges, rank, block_m)
+    r0, r1 = kb * block_m, min(ke * block_m, M)
+    heads = [max(0, min(h, -(-l // block_m) * block_m) - l) for l, h in ranges]
+    H = max(heads)
+    if H == 0:  # every boundary on a block row: nothing to exchange
+        return shard[r0 - lo:r1 - lo] if r1 > r0 else shard[:0], kb, ke
+    mine = torch.zeros((H, N), dtype=shard.dtype, device=shard.device)
+    mine[:heads[rank]] = shard[:heads[rank]]
+    allh = torch.empty((world * H, N), dtype=shard.dtype, device=shard.device)
+    # the rows travel as bytes, which every backend gathers whatever the dtype
+    dist.all_gather_into_tensor(allh.view(torch.uint8), mine.view(torch.uint8), group=group)
+    if r1 <= r0:
+        return shard[:0], kb, ke
+    if r0 >= lo and r1 <= hi:
+        return shard[r0 - lo:r1 - lo], kb, ke
+    out = torch.empty((r1 - r0, N), dtype=shard.dtype, device=shard.device)
+    out[:hi - r0] = shard[r0 - lo:]
+    at = hi  # rows [hi, r1) are the heads of the following ranks, in order
+    for s in range(rank + 1, world):
+        if at >= r1:
+            break
+        l, h = ranges[s]
+        take = min(heads[s], r1 - at)
+        if take > 0:
+            if l != at:
+                raise AssertionError("row ranges leave a gap")
+            out[at - r0:at - r0 + take] = allh[s * H:s * H + take]
+            at += take
+    if at != r1:
+        raise AssertionError(f"rank {rank}: rows {at}..{r1} missing after the exchange")
+    return out, kb, ke
+
+
+def broadcast_quantized(codes, descale, ranges, M: int, N: int,
+                        weight_block_size: Sequence[int] = (128, 128), group=None):
+    """Assemble the whole quantized weight on every rank from each rank's
+    block rows: ``codes`` [rows of block rows kb..ke, N] and ``descale``
+    [ke - kb, gn] of this rank (``exchange_halo``'s block rows).  Each rank
+    broadcasts its part into its place of one [M, N] output (no staging
+    buffer, any part sizes).  Returns ``(codes [M, N], descale [gm, gn])``."""
+    import torch
+    import torch.distributed as dist
+
+    bm, bn = (int(b) for b in weight_block_size)
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    _check_ranges(ranges, M, world)
+    gm, gn = -(-M // bm), -(-N // bn)
+    out_c = torch.empty((M, N), dtype=torch.uint8, device=codes.device)
+    out_s = torch.empty((gm, gn), dtype=torch.float32, device=descale.device)
+    kb, ke = owned_block_rows(ranges, rank, bm)
+    r0, r1 = kb * bm, min(ke * bm, M)
+    if tuple(codes.shape) != (max(0, r1 - r0), N) or tuple(descale.shape) != (ke - kb, gn):
+        raise ValueError(f"rank {rank}: parts {tuple(codes.shape)} / {tuple(descale.shape)} do "
+                         f"not match block rows {kb}..{ke}")
+    if r1 > r0:
+        out_c[r0:r1].copy_(codes.view(torch.uint8))
+        out_s[kb:ke].copy_(descale)
+    for s in range(world):
+        a, b = owned_block_rows(ranges, s, bm)
+        if b > a:
+            src = dist.get_global_rank(group, s) if group is not None else s
+            dist.broadcast(out_c[a * bm:min(b * bm, M)], src=src, group=group)
+            dist.broadcast(out_s[a:b], src=src, group=group)
+    return out_c.view(codes.dtype), out_s
+
+
+def quantize_and_allgather_rows(shard, ranges, M: int,
+                                weight_block_size: Sequence[int] = (128, 128), group=None,
+                                stream=None):
+    """Quantize a weight sharded into any row ranges (``ranges`` = every
+    rank's [lo, hi), e.g. ``row_chunks(M, world)``) and assemble it on every
+    rank: the halo exchange gives each rank whole block rows, the library's
+    CUDA kernel quantizes them, and every rank's codes and descales are
+    broadcast into place.  Returns ``(fp8_data [M, N] float8_e4m3fn,
+    descale [gm, gn] fp32)``, byte for byte ``scaled_fp8_blockwise`` of the
+    whole weight."""
+    import contextlib
+
+    import torch
+
+    from . import scaled_fp8_blockwise
+    block = tuple(int(b) for b in weight_block_size)
+    N = int(shard.shape[-1])
+    ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with ctx:
+        rows, kb, ke = exchange_halo(shard, ranges, M, block[0], group)
+        if rows.shape[0] > 0 and N > 0:
+            codes, descale = scaled_fp8_blockwise(rows, block)
+        else:
+            codes = torch.empty((0, N), dtype=torch.float8_e4m3fn, device=shard.device)
+            descale = torch.empty((ke - kb, -(-N // block[1])), dtype=torch.float32,
+                                  device=shard.device)
+        return broadcast_quantized(codes, descale, ranges, M, N, block, group)

@@ -86,7 +86,9 @@ typedef enum fp8bq_status {
                                      fp8bq_sync_status) */
     FP8BQ_ERR_ALIGN = 8,          /* x not aligned to its element size, or descale not 4-byte
                                      aligned */
-    FP8BQ_ERR_ARG = 9             /* other invalid argument (n_tensors < 0, unknown path) */
+    FP8BQ_ERR_ARG = 9,            /* other invalid argument (n_tensors < 0, unknown path) */
+    FP8BQ_ERR_DEVICE_UNSAFE = 10  /* a kernel returned with a tile copy still in flight
+                                     (reported by fp8bq_sync_status): stop using the GPU */
 } fp8bq_status;
 
 /*
@@ -229,6 +231,18 @@ FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
  * on the current device.  Returns FP8BQ_ERR_DEVICE_TIMEOUT if a kernel of this
  * library gave up a bounded wait since the last check (its outputs are then
  * incomplete), FP8BQ_ERR_DEVICE if the synchronization failed, else FP8BQ_OK.
+ *
+ * FP8BQ_ERR_DEVICE_UNSAFE (it takes precedence over the timeout) if a kernel
+ * returned while one of its tile copies was still in flight: its end-of-kernel
+ * wait for the copies it issued ran out (2 s, which no healthy GPU needs), so
+ * the copy may still land in shared memory that a later kernel of any process
+ * uses; neither the outputs nor any kernel run since can be trusted, and the
+ * process should stop using the GPU.
+ *
+ * The error word is one per device, shared by every stream of the process:
+ * a call reports (and clears) a timeout raised by a kernel on any stream of
+ * the device, not only on `stream`, and whichever call reads it first takes
+ * it.
  */
 FP8BQ_API fp8bq_status fp8bq_sync_status(cudaStream_t stream);
 

@@ -48,7 +48,7 @@ def test_version_and_struct_layout():
 
 
 def test_status_strings():
-    for code in range(10):
+    for code in range(11):
         s = fq.fp8bq_status_string(code)
         assert s.startswith("FP8BQ_")
     assert "unknown" in fq.fp8bq_status_string(1234)

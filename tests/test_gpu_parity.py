@@ -118,6 +118,7 @@ def test_misaligned_pointers(dtype, xoff, yoff):
     ("bf16", 200, 1028, 1036, (64, 64), 1),     # padded rows (poison in the padding)
     ("bf16", 37, 516, None, (1, 128), 1),       # stacked 1x128 blocks, ragged stack
     ("bf16", 130, 4100, None, (128, 128), 3),   # expert stack, 8-byte-aligned strides
+    ("bf16", 129, 4100, None, (128, 128), 3),   # odd experts start 8 bytes past 16
     ("f32", 300, 4098, None, (128, 128), 1),
     ("f32", 200, 1030, 1034, (64, 64), 1),
     ("f32", 37, 514, None, (1, 128), 1),
@@ -142,13 +143,12 @@ def test_half_vector_rows(dtype, M, N, ld, block, batch):
 @pytest.mark.parametrize("shape,block", [
     ((1, 1), (128, 128)), ((5, 5), (128, 128)), ((1, 4096), (1, 128)), ((4096, 1), (128, 128)),
     ((7, 9), (1, 1)), ((256, 256), (256, 256)), ((300, 17), (64, 16)), ((130, 136), (2, 8)),
-    ((64, 4096), (64, 4096)), ((33, 48), (32, 16)),
+    ((64, 4096), (16, 4096)), ((33, 48), (32, 16)),
 ])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_degenerate_shapes_and_blocks(shape, block, dtype):
     M, N = shape
-    if block[0] * block[1] > 65536:
-        pytest.skip("block too large by contract")
+    assert block[0] * block[1] <= 65536     # the largest block the contract allows
     sp = TensorSpec(f"deg.{M}x{N}.b{block}", M, N, block=block, dtype=dtype, seed=71,
                     tensor_id=M * 7919 + N, dist=DIST_STUDENT_T3)
     x = W.materialize(sp)
@@ -305,3 +305,21 @@ def test_many_tensors_in_one_call(path, block):
     outs = run(specs, [buf.data_ptr() + off for off in offs], PATHS[path])
     for sp, x, out in zip(specs, hosts, outs):
         assert_same(sp, out.result(), oracle_expected(sp, x))
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two CUDA devices")
+def test_two_devices_in_one_process():
+    """Kernel attributes and grid sizes are set up per device, so one process
+    may quantize on one GPU, then another, then the first again."""
+    specs = [TensorSpec("dev.tma", 1000, 4096, seed=81, tensor_id=1, dist=DIST_STUDENT_T3),
+             TensorSpec("dev.halves", 1000, 4100, seed=81, tensor_id=2, dist=DIST_STUDENT_T3),
+             TensorSpec("dev.act", 100, 4096, block=(1, 128), seed=81, tensor_id=3)]
+    hosts = [W.materialize(sp) for sp in specs]
+    wants = [oracle_expected(sp, x) for sp, x in zip(specs, hosts)]
+    for dev in (0, 1, 0):
+        with torch.cuda.device(dev):
+            owners = [to_device(x) for x in hosts]
+            outs = run(specs, [p for _, p in owners])
+            for sp, o, w in zip(specs, outs, wants):
+                assert_same(sp, o.result(), w)
+            del owners, outs
