@@ -782,9 +782,12 @@ def run_shard_op(args, specs, lay, x_dev, dev, dist, world, rank, wl_desc) -> No
     def step_ours():
         sqg.run(shards)
 
+    from blockwise_fp8_weight_b200.shard import _coalesced
+
     def step_base():
-        for g, p_ in zip(gathered, pad):
-            tdist.all_gather_into_tensor(g, p_)
+        with _coalesced(None, dev):   # the same coalescing of the gathers as ours
+            for g, p_ in zip(gathered, pad):
+                tdist.all_gather_into_tensor(g.view(torch.uint8), p_.view(torch.uint8))
         st = L.fp8bq_quantize_batched(base_table, len(base_descs), sh)
         if st != 0:
             raise RuntimeError(fq.fp8bq_status_string(st))

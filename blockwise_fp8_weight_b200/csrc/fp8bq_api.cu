@@ -435,6 +435,83 @@ cudaError_t launch_tma_group(int es, const fp8bq_desc *t, const std::vector<int>
     return cudaSuccess;
 }
 
+// ------------------------------------------------------------------ concurrent groups
+//
+// The launch groups of one call (one per kernel variant, dtype and block
+// shape) touch disjoint outputs and only read their inputs, so they may run
+// side by side: the first group runs on the caller's stream, the others on
+// library streams that wait for the caller's stream first, and the caller's
+// stream waits for all of them before anything it enqueues later.  Then one
+// variant's ramp-up and last partial wave overlap another's work instead of
+// adding up.  The streams and events are made once per device and kept (they
+// are not device memory); the fork and join are events, so the call behaves
+// like any sequence of launches on the caller's stream.  A call on a stream
+// that is capturing a CUDA graph launches all its groups on that stream (a
+// library stream forked into one caller's capture would take in another
+// thread's launches until that capture ends).
+#ifndef FP8BQ_GROUP_STREAMS
+#define FP8BQ_GROUP_STREAMS 1
+#endif
+constexpr int kForkStreams = 4;
+
+struct Fork {
+    std::mutex mu;                          // one fork/join at a time per device
+    bool ok = false;
+    cudaStream_t s[kForkStreams] = {};
+    cudaEvent_t start = nullptr, done[kForkStreams] = {};
+};
+
+Fork *fork_of_device() {
+    static PerDevice<Fork *> forks;
+    return forks.get([] {
+        Fork *f = new Fork;
+        f->ok = cudaEventCreateWithFlags(&f->start, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; f->ok && i < kForkStreams; ++i)
+            f->ok = cudaStreamCreateWithFlags(&f->s[i], cudaStreamNonBlocking) == cudaSuccess &&
+                    cudaEventCreateWithFlags(&f->done[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!f->ok) cudaGetLastError();
+        return f;
+    });
+}
+
+// Launch groups 0..n-1 (launch(g, stream)); several groups run concurrently.
+template <typename L>
+fp8bq_status run_groups(size_t n, L &&launch, cudaStream_t stream) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (n > 1 && cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        cs = cudaStreamCaptureStatusActive;  // unknown: do not fork
+    }
+    Fork *f = FP8BQ_GROUP_STREAMS && n > 1 && cs == cudaStreamCaptureStatusNone
+                  ? fork_of_device()
+                  : nullptr;
+    if (f == nullptr || !f->ok) {
+        for (size_t g = 0; g < n; ++g)
+            if (launch(g, stream) != cudaSuccess) return FP8BQ_ERR_DEVICE;
+        return FP8BQ_OK;
+    }
+    std::lock_guard<std::mutex> lock(f->mu);
+    bool ok = cudaEventRecord(f->start, stream) == cudaSuccess;
+    const int aux = (int)std::min<size_t>(n - 1, kForkStreams);
+    for (int i = 0; ok && i < aux; ++i) ok = cudaStreamWaitEvent(f->s[i], f->start, 0) == cudaSuccess;
+    if (!ok) {  // nothing forked: run everything on the caller's stream
+        cudaGetLastError();
+        for (size_t g = 0; g < n; ++g)
+            if (launch(g, stream) != cudaSuccess) return FP8BQ_ERR_DEVICE;
+        return FP8BQ_OK;
+    }
+    for (size_t g = 0; g < n; ++g)  // group g on stream g % (aux + 1); 0 = the caller's
+        if (launch(g, g % (aux + 1) == 0 ? stream : f->s[g % (aux + 1) - 1]) != cudaSuccess)
+            ok = false;
+    // join every forked stream, whatever happened above
+    for (int i = 0; i < aux; ++i)
+        if (cudaEventRecord(f->done[i], f->s[i]) != cudaSuccess ||
+            cudaStreamWaitEvent(stream, f->done[i], 0) != cudaSuccess)
+            ok = false;
+    if (!ok) cudaGetLastError();
+    return ok ? FP8BQ_OK : FP8BQ_ERR_DEVICE;
+}
+
 struct GroupKey {
     Variant v;
     int es, bm, bn;
@@ -490,21 +567,18 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         members[g].push_back(i);
         if (v == Variant::Tma) maps[g].push_back(m);
     }
-    for (size_t g = 0; g < keys.size(); ++g) {
-        cudaError_t e;
+    auto launch = [&](size_t g, cudaStream_t st) -> cudaError_t {
         if (keys[g].v == Variant::Tma)
-            e = members[g].size() <= (size_t)kMaxDescSmall
-                    ? launch_tma_group<kMaxDescSmall>(keys[g].es, table, members[g], maps[g], stream)
-                    : launch_tma_group<kMaxDescTma>(keys[g].es, table, members[g], maps[g], stream);
-        else if (members[g].size() <= (size_t)kMaxDescSmall)
-            e = launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].rows, table,
-                                            members[g], stream);
-        else
-            e = launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].rows, table,
-                                            members[g], stream);
-        if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
-    }
-    return FP8BQ_OK;
+            return members[g].size() <= (size_t)kMaxDescSmall
+                       ? launch_tma_group<kMaxDescSmall>(keys[g].es, table, members[g], maps[g], st)
+                       : launch_tma_group<kMaxDescTma>(keys[g].es, table, members[g], maps[g], st);
+        if (members[g].size() <= (size_t)kMaxDescSmall)
+            return launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].rows, table,
+                                               members[g], st);
+        return launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].rows, table, members[g],
+                                           st);
+    };
+    return run_groups(keys.size(), launch, stream);
 }
 
 // ------------------------------------------------------------------ dequantization
@@ -534,11 +608,8 @@ fp8bq_status check_dequant_desc(const fp8bq_dequant_desc &D, bool *empty) {
 bool dequant_vector_ok(const fp8bq_dequant_desc &D) {
     const int oes = esize_of(D.dtype_out);
     const int64_t obs = D.batch > 1 ? D.out_batch_stride : 0;
-    // the vector kernel numbers its work items (row segments) in 32 bits
-    const uint64_t items = (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll());
     return D.N % 16 == 0 && D.block_n % 16 == 0 && (uintptr_t)D.y_u8 % 16 == 0 &&
-           (uintptr_t)D.out % 16 == 0 && (D.ld_out * oes) % 16 == 0 && (obs * oes) % 16 == 0 &&
-           items < (1ull << 31);
+           (uintptr_t)D.out % 16 == 0 && (D.ld_out * oes) % 16 == 0 && (obs * oes) % 16 == 0;
 }
 
 template <int MAXD>
@@ -552,11 +623,6 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
         p.total = 0;
         while (i < idx.size() && p.n < MAXD) {
             const fp8bq_dequant_desc &D = t[idx[i]];
-            // vector: warp items of 32 x U x 16 codes of a row, numbered in 32 bits
-            const uint64_t items =
-                vector ? (uint64_t)(D.batch * D.M) * (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
-                       : (uint64_t)(D.batch * D.M * D.N);
-            if (vector && p.n > 0 && p.total + items >= (1ull << 32)) break;
             DequantDesc &o = p.d[p.n];
             o.y = D.y_u8;
             o.s = D.descale_f32;
@@ -569,10 +635,11 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.bn = D.block_n;
             o.gm = (int32_t)cdiv(D.M, D.block_m);
             o.gn = (int32_t)cdiv(D.N, D.block_n);
-            o.bm_log2 = is_pow2(D.block_m) ? __builtin_ctz((unsigned)D.block_m) : -1;
-            o.bn_log2 = is_pow2(D.block_n) ? __builtin_ctz((unsigned)D.block_n) : -1;
             o.begin = p.total;
-            o.items = items;
+            // vector: warp items of 32 x 16 codes per row; generic: one element
+            o.items = vector ? (uint64_t)(D.batch * D.M) *
+                                   (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
+                             : (uint64_t)(D.batch * D.M * D.N);
             p.total += o.items;
             ++p.n;
             ++i;
@@ -629,17 +696,18 @@ fp8bq_status run_dequant(const fp8bq_dequant_desc *t, int n, cudaStream_t stream
         const bool v = !generic_only && dequant_vector_ok(t[i]);
         groups[v][t[i].dtype_out == FP8BQ_BF16].push_back(i);
     }
+    std::vector<std::pair<int, int>> used;  // (vector, bf16 output) of each non-empty group
     for (int v = 0; v < 2; ++v)
-        for (int b = 0; b < 2; ++b) {
-            const std::vector<int> &g = groups[v][b];
-            if (g.empty()) continue;
-            const cudaError_t e =
-                g.size() <= (size_t)kMaxDescSmall
-                    ? launch_dequant_group<kMaxDescSmall>(t, g, v, b ? 2 : 4, stream)
-                    : launch_dequant_group<kMaxDescLarge>(t, g, v, b ? 2 : 4, stream);
-            if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
-        }
-    return FP8BQ_OK;
+        for (int b = 0; b < 2; ++b)
+            if (!groups[v][b].empty()) used.emplace_back(v, b);
+    auto launch = [&](size_t k, cudaStream_t st) -> cudaError_t {
+        const int v = used[k].first, b = used[k].second;
+        const std::vector<int> &g = groups[v][b];
+        return g.size() <= (size_t)kMaxDescSmall
+                   ? launch_dequant_group<kMaxDescSmall>(t, g, v, b ? 2 : 4, st)
+                   : launch_dequant_group<kMaxDescLarge>(t, g, v, b ? 2 : 4, st);
+    };
+    return run_groups(used.size(), launch, stream);
 }
 
 // ------------------------------------------------------------------ per-tensor scales

@@ -48,92 +48,85 @@ __device__ __forceinline__ const DequantDesc &find(const DequantPack<MAXD> &p, u
     return p.d[d];
 }
 
-// Vector kernel: a work item is a warp-wide segment of one matrix row, 32
-// lanes x U x 16 codes (U 16-byte loads per lane, all issued before any is
-// used; N and block_n are multiples of 16, so the 16 codes of a load share
-// one descale).  Items are numbered (matrix, row, segment) over the
-// descriptors of a launch (fewer than 2^32 per launch, host-checked) and
-// walked grid-stride by warps; an item costs one or two 32-bit divisions,
-// and the column block of a chunk a shift (power-of-two block_n).
+// Vector kernel: a work item is a warp-wide row segment of 32 x U x 16 codes
+// (U 16-byte loads per lane, all issued before any is used; N and block_n are
+// multiples of 16, so the 16 codes of a load share one descale).  Items are
+// numbered row-major over (matrix, row, segment) and walked grid-stride by
+// warps, so index arithmetic is paid once per segment.
 #ifndef FP8BQ_DQ_UNROLL
-#define FP8BQ_DQ_UNROLL 2
+#define FP8BQ_DQ_UNROLL 2  // measured: 1 -> 4.36, 2 -> 5.41, 4 -> 5.61 TB/s on one layer,
+                           // 4.64 / 5.58 / 5.48 TB/s on the whole weight set
 #endif
+// Measured and dropped: numbering the items in 32 bits with shifts for
+// power-of-two blocks (43.9 M instead of 75.2 M instructions on one layer,
+// yet 142 us instead of 108 us: with the index arithmetic gone, nothing
+// hides the load latency -- long-scoreboard stalls 21 per issue against
+// 3.4), and one warp per whole row (4,199 / 3,889 GB/s against 5,499).
 constexpr int kDqUnroll = FP8BQ_DQ_UNROLL;
-
-__device__ __forceinline__ uint32_t div_p2(uint32_t v, uint32_t d, int log2d) {
-    return log2d >= 0 ? v >> log2d : v / d;
-}
 
 template <int OES, int MAXD>
 __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ DequantPack<MAXD> p) {
     dev::pdl_entry();
     constexpr int U = kDqUnroll;
     const int lane = threadIdx.x & 31;
-    const uint32_t warps = gridDim.x * (blockDim.x >> 5);
-    const uint32_t total = (uint32_t)p.total;
+    const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
     int d = 0;
-    for (uint32_t k = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < total; k += warps) {
+    for (uint64_t k = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < p.total;
+         k += warps) {
         const DequantDesc &a = find(p, k, d);
-        const uint32_t n16 = (uint32_t)(a.N / 16);
-        const uint32_t segs = (n16 + 32 * U - 1) / (32 * U);
-        const uint32_t local = k - (uint32_t)a.begin;
-        const uint32_t row_all = local / segs;  // b * M + r
-        const uint32_t c0 = (local - row_all * segs) * 32 * U + lane;
-        if (c0 >= n16) continue;
-        uint32_t b = 0, r = row_all;
-        if (row_all >= (uint32_t)a.M) {
-            b = row_all / (uint32_t)a.M;
-            r = row_all - b * (uint32_t)a.M;
-        }
-        const uint8_t *src = a.y + (uint64_t)row_all * (uint64_t)a.N;
-        const float *srow =
-            a.s + ((int64_t)b * a.gm + div_p2(r, (uint32_t)a.bm, a.bm_log2)) * a.gn;
-        char *dst = (char *)a.out + ((int64_t)b * a.obs + (int64_t)r * a.ldo) * OES;
-        {
-            uint4 q[U];
+        const int64_t n16 = a.N / 16;
+        const int64_t segs = (n16 + 32 * U - 1) / (32 * U);
+        const int64_t local = (int64_t)(k - a.begin);
+        const int64_t row_all = local / segs;            // b * M + r
+        const int64_t chunk0 = (local - row_all * segs) * 32 * U + lane;
+        if (chunk0 >= n16) continue;
+        const int64_t b = row_all / a.M;
+        const int64_t r = row_all - b * a.M;
+        const uint8_t *src = a.y + row_all * a.N;
+        uint4 q[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t c = c0 + 32 * u;
-                if (c < n16)
-                    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(q[u].x), "=r"(q[u].y), "=r"(q[u].z), "=r"(q[u].w)
-                                 : "l"(src + (uint64_t)c * 16));
+        for (int u = 0; u < U; ++u) {
+            const int64_t chunk = chunk0 + 32 * u;
+            if (chunk < n16)
+                asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(q[u].x), "=r"(q[u].y), "=r"(q[u].z), "=r"(q[u].w)
+                             : "l"(src + chunk * 16));
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t chunk = chunk0 + 32 * u;
+            if (chunk >= n16) break;
+            const int64_t c = chunk * 16;
+            const float s = __ldg(a.s + (b * a.gm + r / a.bm) * a.gn + c / a.bn);
+            uint64_t ss;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
+            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                decode2((uint16_t)(w[j] & 0xffffu), v[4 * j + 0], v[4 * j + 1]);
+                decode2((uint16_t)(w[j] >> 16), v[4 * j + 2], v[4 * j + 3]);
             }
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t c = c0 + 32 * u;
-                if (c >= n16) break;
-                const float s = __ldg(srow + div_p2(c * 16, (uint32_t)a.bn, a.bn_log2));
-                uint64_t ss;
-                asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
-                const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-                float v[16];
+            for (int j = 0; j < 8; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
+            char *dst = (char *)a.out + ((b * a.obs) + r * a.ldo + c) * OES;
+            if constexpr (OES == 2) {
+                uint32_t o[8];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    decode2((uint16_t)(w[j] & 0xffffu), v[4 * j + 0], v[4 * j + 1]);
-                    decode2((uint16_t)(w[j] >> 16), v[4 * j + 2], v[4 * j + 3]);
-                }
+                for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(o[0]),
+                             "r"(o[1]), "r"(o[2]), "r"(o[3])
+                             : "memory");
+                asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16),
+                             "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
+                             : "memory");
+            } else {
 #pragma unroll
-                for (int j = 0; j < 8; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
-                char *o = dst + (uint64_t)c * 16 * OES;
-                if constexpr (OES == 2) {
-                    uint32_t h[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) h[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
-                    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(o), "r"(h[0]),
-                                 "r"(h[1]), "r"(h[2]), "r"(h[3])
+                for (int j = 0; j < 4; ++j)
+                    asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16 * j),
+                                 "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]),
+                                 "f"(v[4 * j + 3])
                                  : "memory");
-                    asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(o + 16),
-                                 "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
-                                 : "memory");
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o + 16 * j),
-                                     "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]),
-                                     "f"(v[4 * j + 3])
-                                     : "memory");
-                }
             }
         }
     }
@@ -166,12 +159,6 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-}  // namespace
-
-int dequant_unroll() { return kDqUnroll; }
-
-namespace {
-
 unsigned dq_grid(uint64_t work) {
     const uint64_t need = (work + 255) / 256;
     const uint64_t cap = (uint64_t)sm_count() * 8;
@@ -179,6 +166,8 @@ unsigned dq_grid(uint64_t work) {
 }
 
 }  // namespace
+
+int dequant_unroll() { return kDqUnroll; }
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st) {

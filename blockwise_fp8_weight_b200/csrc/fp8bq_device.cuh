@@ -133,8 +133,11 @@ __device__ __forceinline__ uint32_t quant_f32x4(uint32_t a, uint32_t b, uint32_t
 //     patterns (for non-negative IEEE values the integer order of the bits is
 //     the numeric order); the running maximum m must have clear sign bits,
 //     as every maximum these functions return has.
+// Measured on B200 (same box, A/B): 1x128 blocks 5765 -> 5972 GB/s, the whole
+// weight set 6421 -> 6456, bf16 4000x4100 5016 -> 5166; 64x64 blocks and
+// one layer unchanged.
 #ifndef FP8BQ_ABSMAX_FMAX
-#define FP8BQ_ABSMAX_FMAX 0
+#define FP8BQ_ABSMAX_FMAX 1
 #endif
 __device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t m, uint32_t w) {
     uint32_t d;

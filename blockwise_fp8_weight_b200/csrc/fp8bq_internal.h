@@ -171,21 +171,19 @@ template <int MAXD>
 cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st);
 
 // Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
-// grouped launch walks the concatenated work items (one matrix row for the
-// vector kernel, one element for the generic one) of all descriptors of a
-// pack.
+// grouped launch walks the concatenated work items (a warp-wide row segment
+// of 32 x 16 codes for the vector kernel, one element for the generic one) of
+// all descriptors of a pack.
 struct DequantDesc {
     const uint8_t *y;   // [batch, M, N] codes
     const float *s;     // [batch, gm, gn] descales
     void *out;          // matrix b at out + b * obs elements, row stride ldo
     int64_t M, N, ldo, obs;
     int32_t bm, bn, gm, gn;
-    int32_t bm_log2;    // log2(bm) if bm is a power of two, else -1
-    int32_t bn_log2;    // log2(bn) if bn is a power of two, else -1
     uint64_t begin;     // first work item of this descriptor
     uint64_t items;     // work items of this descriptor
 };
-static_assert(sizeof(DequantDesc) == 96, "DequantDesc layout");
+static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
 
 template <int MAXD>
 struct DequantPack {

@@ -257,61 +257,57 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             const int64_t xstep = (int64_t)rstep * T.ld * ESIZE;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int r = row0 + i * rstep;
                 uint4 *slot = &stage[(s * V + i) * CTA + threadIdx.x];
                 if constexpr (HALVES) {
+                    // a = this lane's vector in row r; its row starts 8 bytes past a
+                    // 16-byte boundary ("shifted") or on one
+                    const int r = row0 + i * rstep;
+                    const uintptr_t a = (uintptr_t)(src0 + i * xstep);
+                    const bool shifted = ((a - (uintptr_t)(colv * ESIZE)) & 8) != 0;
                     const bool rok = r < T.rows;
-                    const uintptr_t row = (uintptr_t)T.src + (uintptr_t)((int64_t)r * T.ld * ESIZE);
-                    const uintptr_t a = row + (uintptr_t)(colv * ESIZE);
-                    const bool shifted = (row & 8) != 0;
                     const bool lo = rok && colv < T.cols;           // first half in the row
                     const bool hi = rok && colv + VEC / 2 < T.cols;  // second half in the row
+                    // shifted: [a - 8, a + 8), the left lane's second half then our
+                    // first (only the left lane's part where ours lies past the row
+                    // end); else [a, a + 16), or its first half at the row end
+                    const bool left = rok && colv - VEC / 2 < T.cols;
+                    const int n = shifted ? (lo ? 16 : left ? 8 : 0) : (hi ? 16 : lo ? 8 : 0);
                     const char *al = (const char *)(a & ~(uintptr_t)15);
-                    if (shifted) {
-                        // [a - 8, a + 8): the left lane's second half, then ours; only
-                        // the left lane's part when ours lies beyond the row end
-                        const bool left = rok && colv - VEC / 2 < T.cols;
-                        const int n = lo ? 16 : left ? 8 : 0;
-                        dev::cp_async_16_n(slot, n ? al : safe(T), n);
-                        if (last_lane)  // our second half, [a + 8, a + 16)
-                            dev::cp_async_16_n(&extra[(s * V + i) * XR + xrow],
-                                               hi ? al + 16 : safe(T), hi ? 8 : 0);
-                    } else {
-                        const int n = hi ? 16 : lo ? 8 : 0;
-                        dev::cp_async_16_n(slot, n ? al : safe(T), n);
-                    }
+                    dev::cp_async_16_n(slot, n ? al : safe(T), n);
+                    if (shifted && last_lane)  // our second half, [a + 8, a + 16)
+                        dev::cp_async_16_n(&extra[(s * V + i) * XR + xrow], hi ? al + 16 : safe(T),
+                                           hi ? 8 : 0);
                 } else {
+                    const int r = row0 + i * rstep;
                     const bool ok = full || (r < T.rows && colv < T.cols);
                     dev::cp_async_16(slot, ok ? src0 + i * xstep : T.src, ok);
                 }
             }
             dev::cp_async_commit();
         };
-        // Read this thread's vectors of stage s (HALVES: after every lane's
-        // copies have landed, reassembled across the slots of a shifted row).
+        // Read this thread's vectors of stage s.  HALVES: a shifted row's
+        // vector is the second half of this lane's slot followed by the first
+        // half of lane cv + 1's slot, fetched by shuffle (the row's last lane
+        // reads its extra slot): every lane reads only what it copied itself.
         auto fetch = [&](int s, const Tile &T, uint4 (&R)[V]) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
             if constexpr (HALVES) {
-                // the copies of the row's other lanes (same team, same warp) are visible
-                __syncwarp(shfl_mask);
+                const uintptr_t a0 = (uintptr_t)T.src + (uintptr_t)((int64_t)row0 * T.ld * ESIZE);
+                const uintptr_t xstep = (uintptr_t)((int64_t)rstep * T.ld * ESIZE);
+                constexpr int W = TEAM >= 32 ? 32 : TEAM;
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
-                    const int r = row0 + i * rstep;
-                    const uint4 *slot = &stage[(s * V + i) * CTA + threadIdx.x];
-                    const bool shifted =
-                        (((uintptr_t)T.src + (uintptr_t)((int64_t)r * T.ld * ESIZE)) & 8) != 0;
-                    if (shifted) {
-                        const uint2 lo = dev::lds_v2(reinterpret_cast<const char *>(slot) + 8);
-                        const uint2 up = dev::lds_v2(last_lane ? (const void *)&extra[(s * V + i) * XR + xrow]
-                                                               : (const void *)(slot + 1));
-                        R[i] = make_uint4(lo.x, lo.y, up.x, up.y);
-                    } else {
-                        R[i] = *slot;
+                    const bool shifted = ((a0 + i * xstep) & 8) != 0;
+                    uint32_t ux = __shfl_down_sync(shfl_mask, R[i].x, 1, W);
+                    uint32_t uy = __shfl_down_sync(shfl_mask, R[i].y, 1, W);
+                    if (shifted && last_lane) {
+                        const uint2 e = dev::lds_v2(&extra[(s * V + i) * XR + xrow]);
+                        ux = e.x;
+                        uy = e.y;
                     }
+                    if (shifted) R[i] = make_uint4(R[i].z, R[i].w, ux, uy);
                 }
-                __syncwarp(shfl_mask);  // every lane has read the stage before any refills it
-            } else {
-#pragma unroll
-                for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
             }
         };
         Tile Ts[S];

@@ -90,14 +90,29 @@ def gather_buffers(M: int, N: int, weight_block_size: Sequence[int], world: int,
 
 def _gather_in_place(buf: GatherBuffers, rank: int, group) -> None:
     """All-gather every rank's slot into every rank's buffer (each rank sends
-    its own slot of the output, so nothing is staged)."""
+    its own slot of the output, so nothing is staged); descales travel as
+    bytes, so every gather of a weight has one dtype."""
+    import torch
     import torch.distributed as dist
     bm = buf.block[0]
     per_c, per_s = buf.rows, buf.rows // bm
     dist.all_gather_into_tensor(buf.codes, buf.codes[rank * per_c:(rank + 1) * per_c],
                                 group=group)
-    dist.all_gather_into_tensor(buf.descale, buf.descale[rank * per_s:(rank + 1) * per_s],
-                                group=group)
+    sb = buf.descale.view(torch.uint8)
+    dist.all_gather_into_tensor(sb, buf.descale[rank * per_s:(rank + 1) * per_s]
+                                .view(torch.uint8), group=group)
+
+
+def _coalesced(group, device):
+    """One NCCL group launch for the gathers issued inside (other backends:
+    one call each)."""
+    import contextlib
+
+    import torch.distributed as dist
+    if dist.get_backend(group) == "nccl":
+        from torch.distributed.distributed_c10d import _coalescing_manager
+        return _coalescing_manager(group=group, device=device)
+    return contextlib.nullcontext()
 
 
 def _check_shard(what, rank, shape, want) -> None:
@@ -207,7 +222,10 @@ class ShardedQuantGather:
         self.shapes = [(int(M), int(N)) for M, N in shapes]
         self.ranges = [shard_rows(M, self.world, self.block[0])[self.rank]
                        for M, _ in self.shapes]
+        self.device = dev
         self.bufs = [gather_buffers(M, N, self.block, self.world, dev) for M, N in self.shapes]
+        self._table = None  # descriptor table of the last shards, reused while they stay put
+        self._key = None
 
     def run(self, shards, stream=None):
         import contextlib
@@ -219,18 +237,25 @@ class ShardedQuantGather:
             raise ValueError(f"{len(shards)} shards for {len(self.shapes)} weights")
         ctx = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
         with ctx:
-            descs = []
-            for x, (M, N), (lo, hi), buf in zip(shards, self.shapes, self.ranges, self.bufs):
-                _check_shard("the shard is", self.rank, x.shape, (hi - lo, N))
-                if hi > lo and N > 0:
-                    yc, sc = buf.slot(self.rank, lo, hi)
-                    descs.append(make_desc(x, yc, sc, self.block))
-            if descs:
-                check(fp8bq_quantize_batched(descs), "ShardedQuantGather")
+            key = tuple((int(x.data_ptr()), tuple(x.shape), tuple(x.stride()), x.dtype)
+                        for x in shards)
+            if key != self._key:
+                descs = []
+                for x, (M, N), (lo, hi), buf in zip(shards, self.shapes, self.ranges, self.bufs):
+                    _check_shard("the shard is", self.rank, x.shape, (hi - lo, N))
+                    if hi > lo and N > 0:
+                        yc, sc = buf.slot(self.rank, lo, hi)
+                        descs.append(make_desc(x, yc, sc, self.block))
+                self._table = descs
+                self._key = key
+            if self._table:
+                check(fp8bq_quantize_batched(self._table), "ShardedQuantGather")
+            with _coalesced(self.group, self.device):
+                for (M, N), buf in zip(self.shapes, self.bufs):
+                    if M > 0 and N > 0:
+                        _gather_in_place(buf, self.rank, self.group)
             out = []
-            for (M, N), buf in zip(self.shapes, self.bufs):
-                if M > 0 and N > 0:
-                    _gather_in_place(buf, self.rank, self.group)
+            for buf in self.bufs:
                 y, s = buf.whole()
                 out.append((y.view(torch.float8_e4m3fn), s))
             return out

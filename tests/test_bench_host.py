@@ -121,3 +121,21 @@ def test_shape_workload_and_launch_count():
     qwen = W.qwen3_8b_model()
     lay = bench.Layout(qwen)
     assert bench.count_launches(bench.build_descs(qwen, lay, 1 << 40, 1 << 41, 1 << 42)) == 2
+
+
+def test_traffic_record_lookup(tmp_path, monkeypatch):
+    """roofline.traffic comes from a record taken on the current TMA kernel
+    sources only, per launch, with the record's note on how it was obtained."""
+    dig = bench.kernel_digest()
+    f = tmp_path / "traffic.txt"
+    f.write_text("# comment line\n"
+                 f"qwen3_8b_model auto {dig} 2000000000 scaled from qwen3_8b_layer x 36.0\n"
+                 f"moe_layer auto {dig} 1800000000\n"
+                 "qwen3_8b_layer auto 0123456789abcdef 579000000 captured\n")
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(f))
+    assert bench.traffic_for("qwen3_8b_model", "auto", 2) == (1e9, "scaled from qwen3_8b_layer x 36.0")
+    assert bench.traffic_for("moe_layer", "auto", 1) == (1.8e9, "captured")
+    assert bench.traffic_for("qwen3_8b_layer", "auto", 1) == (None, None)   # other sources
+    assert bench.traffic_for("qwen3_8b_model", "tma", 2) == (None, None)
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(tmp_path / "missing.txt"))
+    assert bench.traffic_for("qwen3_8b_model", "auto", 2) == (None, None)

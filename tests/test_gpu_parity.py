@@ -323,3 +323,55 @@ def test_two_devices_in_one_process():
             for sp, o, w in zip(specs, outs, wants):
                 assert_same(sp, o.result(), w)
             del owners, outs
+
+
+def test_concurrent_groups_keep_stream_order(edge_case):
+    """A call whose tensors take several kernel variants runs its launch
+    groups side by side on library streams forked from the caller's stream and
+    joined back: work the caller enqueues next on its stream (here a copy of
+    every output, with no host synchronization in between) sees every byte."""
+    from tests.gpu_util import Outputs
+    case = edge_case
+    outs = [Outputs(sp) for sp in case.specs]
+    descs = [o.desc(p) for o, p in zip(outs, case.ptrs)]
+    s = torch.cuda.Stream()
+    for _ in range(3):
+        for o in outs:                                   # stale bytes the copies must not see
+            o.y.view.fill_(0x7F)
+            o.s.view.fill_(0xFF)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            assert fq.fp8bq_quantize_batched(descs, stream=s) == fq.FP8BQ_OK
+            copies = [(o.y.view.clone(), o.s.view.clone()) for o in outs]
+        s.synchronize()
+        assert fq.fp8bq_sync_status(s) == fq.FP8BQ_OK
+        for sp, (yc, sc), w in zip(case.specs, copies, case.want):
+            gm, gn = sp.grid
+            assert_same(sp, (yc.cpu().numpy().reshape(sp.batch, sp.M, sp.N),
+                             sc.cpu().numpy().view(np.float32).reshape(sp.batch, gm, gn)), w)
+
+
+def test_mixed_variant_call_in_a_cuda_graph(edge_case):
+    """Under graph capture the launch groups of a call stay on the capturing
+    stream; replays write the oracle's bytes."""
+    from tests.gpu_util import Outputs
+    case = edge_case
+    outs = [Outputs(sp) for sp in case.specs]
+    descs = (fq.fp8bq_desc * len(outs))(*[o.desc(p) for o, p in zip(outs, case.ptrs)])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        assert fq.fp8bq_quantize_batched(descs, stream=s) == fq.FP8BQ_OK   # warm-up
+    s.synchronize()
+    for o in outs:
+        o.y.view.fill_(0)
+        o.s.view.fill_(0)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        st = fq.fp8bq_quantize_batched(descs, stream=s)
+    assert st == fq.FP8BQ_OK
+    g.replay()
+    torch.cuda.synchronize()
+    assert fq.fp8bq_sync_status() == fq.FP8BQ_OK
+    for sp, o, w in zip(case.specs, outs, case.want):
+        assert_same(sp, o.result(), w)
