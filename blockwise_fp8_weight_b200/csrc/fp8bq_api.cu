@@ -158,23 +158,6 @@ bool halves_aligned(const fp8bq_desc &D) {
     return true;
 }
 
-// Row class of a tensor on the vector kernel: whole 16-byte vectors; or
-// 8-byte aligned rows loaded into registers; or (FP8BQ_HALVES_RING) the same
-// rows through the shifted cp.async ring (x itself 16-byte aligned, so no
-// copy starts before the tensor, and enough vectors per block row for its
-// extra slots).  Measured on B200 (bf16 4000x4100, 16 such tensors in one
-// call): registers 5270 GB/s, shifted ring 3784 GB/s -- the ring is off.
-#ifndef FP8BQ_HALVES_RING
-#define FP8BQ_HALVES_RING 0
-#endif
-Rows rows_of(const fp8bq_desc &D) {
-    if (vector_aligned(D)) return Rows::Aligned16;
-    const int vec = 16 / esize_of(D.dtype_in);
-    if (FP8BQ_HALVES_RING && (uintptr_t)D.x % 16 == 0 && D.block_n / vec >= kHalvesMinVpr)
-        return Rows::HalvesRing;
-    return Rows::HalvesRegs;
-}
-
 Variant vector_variant(const fp8bq_desc &D) {
     for (Variant v : {Variant::VecT16, Variant::VecT64, Variant::VecTBig})
         if (vector_fits(D, v)) return v;
@@ -382,7 +365,7 @@ void pack_header(DescPack<MAXD> &p) {
 // Launch one group (same variant, dtype and, for vector/TMA, block shape) in
 // chunks that fit the parameter pack and keep the tile count below 2^31.
 template <int MAXD>
-cudaError_t launch_group(Variant v, int es, Rows rows, const fp8bq_desc *t,
+cudaError_t launch_group(Variant v, int es, bool halves, const fp8bq_desc *t,
                          const std::vector<int> &idx, cudaStream_t st) {
     static thread_local DescPack<MAXD> p;  // large: keep it off the stack
     size_t i = 0;
@@ -398,7 +381,7 @@ cudaError_t launch_group(Variant v, int es, Rows rows, const fp8bq_desc *t,
             ++i;
         }
         const cudaError_t e = v == Variant::Generic ? launch_generic<MAXD>(es, p, st)
-                                                    : launch_vector<MAXD>(v, es, rows, p, st);
+                                                    : launch_vector<MAXD>(v, es, halves, p, st);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
@@ -515,9 +498,9 @@ fp8bq_status run_groups(size_t n, L &&launch, cudaStream_t stream) {
 struct GroupKey {
     Variant v;
     int es, bm, bn;
-    Rows rows;
+    bool halves;
     bool operator==(const GroupKey &o) const {
-        return v == o.v && es == o.es && bm == o.bm && bn == o.bn && rows == o.rows;
+        return v == o.v && es == o.es && bm == o.bm && bn == o.bn && halves == o.halves;
     }
 };
 
@@ -553,10 +536,9 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         // vector / TMA launches need one block shape; generic ones only one
         // size class (CTA per block for >= 2048 elements, else warp per block)
         const bool big = (int64_t)D.block_m * D.block_n >= 2048;
-        const Rows rows =
-            v != Variant::Generic && v != Variant::Tma ? rows_of(D) : Rows::Aligned16;
+        const bool halves = v != Variant::Generic && v != Variant::Tma && !vector_aligned(D);
         GroupKey k{v, esize_of(D.dtype_in), v == Variant::Generic ? (int)big : D.block_m,
-                   v == Variant::Generic ? 0 : D.block_n, rows};
+                   v == Variant::Generic ? 0 : D.block_n, halves};
         size_t g = 0;
         while (g < keys.size() && !(keys[g] == k)) ++g;
         if (g == keys.size()) {
@@ -573,10 +555,10 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
                        ? launch_tma_group<kMaxDescSmall>(keys[g].es, table, members[g], maps[g], st)
                        : launch_tma_group<kMaxDescTma>(keys[g].es, table, members[g], maps[g], st);
         if (members[g].size() <= (size_t)kMaxDescSmall)
-            return launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].rows, table,
+            return launch_group<kMaxDescSmall>(keys[g].v, keys[g].es, keys[g].halves, table,
                                                members[g], st);
-        return launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].rows, table, members[g],
-                                           st);
+        return launch_group<kMaxDescLarge>(keys[g].v, keys[g].es, keys[g].halves, table,
+                                           members[g], st);
     };
     return run_groups(keys.size(), launch, stream);
 }

@@ -195,22 +195,6 @@ __device__ __forceinline__ void cp_async_16(void *smem_dst, const void *src, boo
                  "l"(src), "r"(ok ? 16 : 0)
                  : "memory");
 }
-// The same with the number of bytes to read given (0, 8 or 16; the rest of
-// the 16 is zero-filled); src 16-byte aligned.
-__device__ __forceinline__ void cp_async_16_n(void *smem_dst, const void *src, int src_bytes) {
-    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(smem_addr(smem_dst)),
-                 "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-// 8-byte shared-memory load (8-byte aligned address).
-__device__ __forceinline__ uint2 lds_v2(const void *p) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];"
-                 : "=r"(v.x), "=r"(v.y)
-                 : "r"(smem_addr(p))
-                 : "memory");
-    return v;
-}
 __device__ __forceinline__ void cp_async_commit() {
     asm volatile("cp.async.commit_group;" ::: "memory");
 }

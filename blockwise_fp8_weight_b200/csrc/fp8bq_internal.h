@@ -147,21 +147,11 @@ enum class Variant : int {
     Tma = 4,
 };
 
-// Row alignment classes of the vector kernel (uniform per launch).
-enum class Rows : int {
-    Aligned16 = 0,   // 16-byte aligned rows: cp.async ring of whole vectors
-    HalvesRing = 1,  // 8-byte aligned rows, x 16-byte aligned, >= kHalvesMinVpr vectors
-                     // per block row: cp.async ring of aligned 16-byte copies, shifted rows
-                     // reassembled in shared memory
-    HalvesRegs = 2,  // other 8-byte aligned rows: two 8-byte loads per vector into registers
-};
-// Fewest 16-byte vectors per block row for Rows::HalvesRing (sizes its extra slots).
-constexpr int kHalvesMinVpr = 8;
-
 // Launchers (vector and generic: fp8bq_kernels.cu; TMA: fp8bq_tma.cu).  Each
 // returns cudaSuccess or the launch error.
+// halves: rows only 8-byte aligned (each 16-byte vector moved as two halves)
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, Rows rows, const DescPack<MAXD> &p,
+cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
                           cudaStream_t st);
 template <int MAXD>
 cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st);

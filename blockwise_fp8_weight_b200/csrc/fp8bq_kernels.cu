@@ -43,27 +43,29 @@ namespace fp8bq {
 // Reduce-scatter of 8 per-lane maxima over an aligned team of 16 lanes:
 // three halving exchange steps (xor 8, 4, 2) and one full step (xor 1).
 // Afterwards team lane q holds the team-wide max of slot 4*b3 + 2*b2 + b1
-// (b_k = bit k of q), i.e. slot q / 2; 8 shuffles instead of 32.
+// (b_k = bit k of q), i.e. slot q / 2; 8 shuffles instead of 32.  `merge`
+// combines two running maxima (packed bf16 magnitudes or fp32 ones).
+template <typename Merge>
 __device__ __forceinline__ uint32_t reduce_scatter8x16(const uint32_t (&m)[8], uint32_t mask,
-                                                      int q) {
+                                                      int q, Merge merge) {
     const bool h3 = q & 8, h2 = q & 4, h1 = q & 2;
     uint32_t a[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t send = h3 ? m[j] : m[j + 4];
         const uint32_t keep = h3 ? m[j + 4] : m[j];
-        a[j] = max(keep, __shfl_xor_sync(mask, send, 8));
+        a[j] = merge(keep, __shfl_xor_sync(mask, send, 8));
     }
     uint32_t b[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const uint32_t send = h2 ? a[j] : a[j + 2];
         const uint32_t keep = h2 ? a[j + 2] : a[j];
-        b[j] = max(keep, __shfl_xor_sync(mask, send, 4));
+        b[j] = merge(keep, __shfl_xor_sync(mask, send, 4));
     }
     const uint32_t send = h1 ? b[0] : b[1];
-    uint32_t c = max(h1 ? b[1] : b[0], __shfl_xor_sync(mask, send, 2));
-    return max(c, __shfl_xor_sync(mask, c, 1));
+    uint32_t c = merge(h1 ? b[1] : b[0], __shfl_xor_sync(mask, send, 2));
+    return merge(c, __shfl_xor_sync(mask, c, 1));
 }
 
 // vec_quant_store for a lane's 16 bytes held as two 8-byte halves (rows that
@@ -100,27 +102,21 @@ __device__ __forceinline__ void vec_quant_store_halves(const uint4 &v, uint64_t 
 // geometry, each 16-byte vector moved as two 8-byte halves; a half beyond
 // the row end reads as zeros (no effect on the absmax) and is not stored.
 //
-// S > 0: the loads go through a ring of S stages in shared memory (cp.async,
-// 16-byte copies), S - 1 tiles in flight while one is reduced and stored;
-// slot i of thread t of stage s is stage[(s * V + i) * CTA + t], so the
-// slots of the vpr lanes of a block row are 16 * vpr contiguous bytes.
-//   16-byte aligned rows: each lane copies its own vector.
-//   HALVES (rows 8-byte aligned, x 16-byte aligned, vpr >= 8): in a row
-//   that starts 8 bytes past a 16-byte boundary ("shifted"), lane cv copies
-//   the aligned 16 bytes that begin 8 bytes before its vector (the tail of
-//   its left neighbour's vector, then its own first half), and its vector is
-//   read back from shared memory 8 bytes into its slot: its first half, then
-//   the head of lane cv + 1's slot; the last lane of the row copies that
-//   second half into a per-row extra slot.  Every copy starts on a 16-byte
-//   boundary; bytes beyond the row end are zero-filled, not read.
-// S == 0 (HALVES, other cases): two register sets, the next tile loaded
-// straight into registers (two 8-byte loads per vector) while the current one
-// is processed.
+// S > 0 (16-byte aligned rows): the loads go through a private ring of S
+// stages per thread in shared memory (cp.async), S - 1 tiles in flight while
+// one is reduced and stored.  S == 0 (HALVES): two register sets, the next
+// tile loaded while the current one is processed.  Measured and dropped for
+// HALVES: a ring of 8-byte cp.async copies (4.10 against 4.38-4.65 TB/s), and
+// a ring of 16-byte copies from the aligned addresses of rows that start 8
+// bytes past a 16-byte boundary, reassembled in shared memory or by shuffle
+// (2971-3505 against 5016-5293 GB/s on bf16 4000x4100: divergent even/odd
+// rows within a warp, 40 % bank conflicts or a shuffle pair per vector).
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, int S>
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     dev::pdl_entry();
     static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
+    static_assert(!(HALVES && S > 0), "the cp.async ring takes 16-byte vectors only");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
     constexpr int WPT = TEAM >= 32 ? TEAM / 32 : 1;
@@ -152,9 +148,10 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     // Every slot of every lane of the team lies inside the tile (the same for
     // the whole team): the interior tiles skip the per-vector bounds checks.
     auto is_full = [&](const Tile &T) { return T.rows >= V * rstep && T.cols >= vpr * VEC; };
-    // Quantize and store slot i of every lane for i < NB (the slots of blocks
-    // inside the matrix), with the reciprocal rr(i).
-    auto store_all = [&](const uint4 (&R)[V], const Tile &T, int nb, auto rr_of) {
+    // Quantize and store slot i of every lane with the reciprocal rr(i): every
+    // slot inside the tile (a slot of a block below the matrix lies below it
+    // too, so the row check covers both).
+    auto store_all = [&](const uint4 (&R)[V], const Tile &T, auto rr_of) {
         uint8_t *dst = T.dst + (int64_t)row0 * T.ldy + colv;
         const int64_t ystep = (int64_t)rstep * T.ldy;
         if (is_full(T)) {
@@ -163,11 +160,9 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         } else {
             const bool hi = hi_ok(T);
 #pragma unroll
-            for (int i = 0; i < V; ++i) {
-                if (i >= nb) break;
+            for (int i = 0; i < V; ++i)
                 if (row0 + i * rstep < T.rows && colv < T.cols)
                     store(R[i], rr_of(i), dst + i * ystep, hi);
-            }
         }
     };
 
@@ -193,23 +188,27 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
       if constexpr (TEAM == 16 && V == 8) {  // the only stacked-block instantiation
         const int bm = p.d[0].bm;
+        // running maxima stay packed (two bf16 magnitudes per word) through the
+        // reduce-scatter; only the one this lane ends with is unpacked
         uint32_t m[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const uint4 one[1] = {R[i]};
-            m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
-        }
+        for (int i = 0; i < V; ++i) m[i] = vec_absmax<ESIZE>(R[i]);
         // lane q ends with the max of slot q / 2, computes its scale, and the
         // reciprocal of slot i is fetched from lane 2 i of the team
-        const uint32_t mq = reduce_scatter8x16(m, shfl_mask, lane);
+        const uint32_t mq = absmax_to_f32_bits<ESIZE>(reduce_scatter8x16(
+            m, shfl_mask, lane, [](uint32_t a, uint32_t b) {
+                if constexpr (ESIZE == 2)
+                    return dev::absmax_bf16x2(a, b);
+                else
+                    return dev::absmax_f32(a, b);
+            }));
         float s_mine, r_mine;
         dev::block_scale(mq, kEps, s_mine, r_mine);
         const int base = (threadIdx.x & 31) & ~(TEAM - 1);
         float r[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + 2 * i);
-        // slots of blocks below the matrix are neither quantized nor stored
-        store_all(R, T, (T.rows + bm - 1) / bm, [&](int i) { return dev::splat2(r[i]); });
+        store_all(R, T, [&](int i) { return dev::splat2(r[i]); });
         const int slot = lane >> 1;
         if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
       }
@@ -235,80 +234,24 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         float s, r;
         dev::block_scale(m, kEps, s, r);
         const uint64_t r2 = dev::splat2(r);
-        store_all(R, T, V, [&](int) { return r2; });
+        store_all(R, T, [&](int) { return r2; });
         if (lane == 0) *T.sdst = s;
     };
 
     if constexpr (S > 0) {
         extern __shared__ __align__(1024) uint8_t ring[];  // dynamic shared memory
         uint4 *const stage = reinterpret_cast<uint4 *>(ring);  // [S][V][CTA] 16-byte vectors
-        // HALVES: [S][V][CTA / kHalvesMinVpr] extra slots, one per row of a row step
-        uint4 *const extra = stage + S * V * CTA;
-        constexpr int XR = CTA / kHalvesMinVpr;
-        const bool last_lane = cv == vpr - 1;
-        const int xrow = threadIdx.x / vpr;  // this thread's row within the CTA's row step
-        // an aligned source for copies that read nothing (x is 16-byte aligned)
-        auto safe = [](const Tile &T) {
-            return (const char *)((uintptr_t)T.src & ~(uintptr_t)15);
-        };
         auto issue = [&](int s, const Tile &T) {
             const bool full = is_full(T);
             const char *src0 = T.src + ((int64_t)row0 * T.ld + colv) * ESIZE;
             const int64_t xstep = (int64_t)rstep * T.ld * ESIZE;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                uint4 *slot = &stage[(s * V + i) * CTA + threadIdx.x];
-                if constexpr (HALVES) {
-                    // a = this lane's vector in row r; its row starts 8 bytes past a
-                    // 16-byte boundary ("shifted") or on one
-                    const int r = row0 + i * rstep;
-                    const uintptr_t a = (uintptr_t)(src0 + i * xstep);
-                    const bool shifted = ((a - (uintptr_t)(colv * ESIZE)) & 8) != 0;
-                    const bool rok = r < T.rows;
-                    const bool lo = rok && colv < T.cols;           // first half in the row
-                    const bool hi = rok && colv + VEC / 2 < T.cols;  // second half in the row
-                    // shifted: [a - 8, a + 8), the left lane's second half then our
-                    // first (only the left lane's part where ours lies past the row
-                    // end); else [a, a + 16), or its first half at the row end
-                    const bool left = rok && colv - VEC / 2 < T.cols;
-                    const int n = shifted ? (lo ? 16 : left ? 8 : 0) : (hi ? 16 : lo ? 8 : 0);
-                    const char *al = (const char *)(a & ~(uintptr_t)15);
-                    dev::cp_async_16_n(slot, n ? al : safe(T), n);
-                    if (shifted && last_lane)  // our second half, [a + 8, a + 16)
-                        dev::cp_async_16_n(&extra[(s * V + i) * XR + xrow], hi ? al + 16 : safe(T),
-                                           hi ? 8 : 0);
-                } else {
-                    const int r = row0 + i * rstep;
-                    const bool ok = full || (r < T.rows && colv < T.cols);
-                    dev::cp_async_16(slot, ok ? src0 + i * xstep : T.src, ok);
-                }
+                const bool ok = full || (row0 + i * rstep < T.rows && colv < T.cols);
+                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], ok ? src0 + i * xstep : T.src,
+                                 ok);
             }
             dev::cp_async_commit();
-        };
-        // Read this thread's vectors of stage s.  HALVES: a shifted row's
-        // vector is the second half of this lane's slot followed by the first
-        // half of lane cv + 1's slot, fetched by shuffle (the row's last lane
-        // reads its extra slot): every lane reads only what it copied itself.
-        auto fetch = [&](int s, const Tile &T, uint4 (&R)[V]) {
-#pragma unroll
-            for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
-            if constexpr (HALVES) {
-                const uintptr_t a0 = (uintptr_t)T.src + (uintptr_t)((int64_t)row0 * T.ld * ESIZE);
-                const uintptr_t xstep = (uintptr_t)((int64_t)rstep * T.ld * ESIZE);
-                constexpr int W = TEAM >= 32 ? 32 : TEAM;
-#pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    const bool shifted = ((a0 + i * xstep) & 8) != 0;
-                    uint32_t ux = __shfl_down_sync(shfl_mask, R[i].x, 1, W);
-                    uint32_t uy = __shfl_down_sync(shfl_mask, R[i].y, 1, W);
-                    if (shifted && last_lane) {
-                        const uint2 e = dev::lds_v2(&extra[(s * V + i) * XR + xrow]);
-                        ux = e.x;
-                        uy = e.y;
-                    }
-                    if (shifted) R[i] = make_uint4(R[i].z, R[i].w, ux, uy);
-                }
-            }
         };
         Tile Ts[S];
         uint32_t tn = t;  // next tile to issue; t: next tile to process
@@ -333,7 +276,8 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
                 }
                 dev::cp_async_wait<S - 1>();  // this thread's copies of stage s have landed
                 uint4 R[V];
-                fetch(s, Ts[s], R);
+#pragma unroll
+                for (int i = 0; i < V; ++i) R[i] = stage[(s * V + i) * CTA + threadIdx.x];
                 process(R, Ts[s], it++);  // consumes R: the stage is free again
                 if (tn < p.total_tiles) {
                     Ts[s] = walk.next(tn);
@@ -470,14 +414,10 @@ __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ Des
 
 namespace {
 
-// RING: the cp.async ring (16-byte aligned rows, or HALVES rows that the
-// shifted ring can take); else the register path (HALVES only).
-template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, bool RING>
+template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
-    static_assert(RING || HALVES, "16-byte aligned rows always take the ring");
-    constexpr int S = !RING ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
-    constexpr size_t smem =
-        (size_t)S * V * CTA * 16 + (HALVES ? (size_t)S * V * (CTA / kHalvesMinVpr) * 16 : 0);
+    constexpr int S = HALVES ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
+    constexpr size_t smem = (size_t)S * V * CTA * 16;
     auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES, S>;
     static PerDevice<KernelSetup> setup;
     const KernelSetup ks = setup.get([&] { return setup_kernel(kern, CTA, smem); });
@@ -487,31 +427,28 @@ cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
 }
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD>
-cudaError_t launch_vector_t(Rows rows, const DescPack<MAXD> &p, cudaStream_t st) {
-    switch (rows) {
-        case Rows::Aligned16: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, false, true>(p, st);
-        case Rows::HalvesRing: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true, true>(p, st);
-        default: return launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true, false>(p, st);
-    }
+cudaError_t launch_vector_t(bool halves, const DescPack<MAXD> &p, cudaStream_t st) {
+    return halves ? launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, true>(p, st)
+                  : launch_vector_h<ESIZE, TEAM, V, CTA, G, MAXD, false>(p, st);
 }
 
 }  // namespace
 
 template <int MAXD>
-cudaError_t launch_vector(Variant v, int esize, Rows rows, const DescPack<MAXD> &p,
+cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD> &p,
                           cudaStream_t st) {
     if (esize == 2) {
         switch (v) {
-            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(rows, p, st);
-            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(rows, p, st);
-            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(rows, p, st);
+            case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(halves, p, st);
+            case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(halves, p, st);
+            case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(halves, p, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (v) {
-        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(rows, p, st);
-        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(rows, p, st);
-        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(rows, p, st);
+        case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(halves, p, st);
+        case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(halves, p, st);
+        case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(halves, p, st);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -536,10 +473,10 @@ cudaError_t launch_generic(int esize, const DescPack<MAXD> &p, cudaStream_t st) 
     return e;
 }
 
-template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, Rows,
+template cudaError_t launch_vector<kMaxDescSmall>(Variant, int, bool,
                                                   const DescPack<kMaxDescSmall> &,
                                                   cudaStream_t);
-template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, Rows,
+template cudaError_t launch_vector<kMaxDescLarge>(Variant, int, bool,
                                                   const DescPack<kMaxDescLarge> &,
                                                   cudaStream_t);
 template cudaError_t launch_generic<kMaxDescSmall>(int, const DescPack<kMaxDescSmall> &,

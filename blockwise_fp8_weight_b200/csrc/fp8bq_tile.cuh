@@ -122,10 +122,22 @@ struct TileCursor {
     }
 };
 
+// absmax bits of one 16-byte vector: a tree of three maxima.
+template <int ESIZE>
+__device__ __forceinline__ uint32_t vec_absmax(const uint4 &v) {
+    if constexpr (ESIZE == 2)
+        return dev::absmax_bf16x2(dev::absmax_bf16x2(v.x & 0x7fff7fffu, v.y),
+                                  dev::absmax_bf16x2(v.z & 0x7fff7fffu, v.w));
+    else
+        return dev::absmax_f32(dev::absmax_f32(v.x & 0x7fffffffu, v.y),
+                               dev::absmax_f32(v.z & 0x7fffffffu, v.w));
+}
+
 // absmax bits of V 16-byte vectors: four independent running maxima (one per
 // 32-bit lane of the vectors) so the max chains overlap, merged at the end.
 template <int ESIZE, int V>
 __device__ __forceinline__ uint32_t tile_absmax(const uint4 (&R)[V]) {
+    if constexpr (V == 1) return vec_absmax<ESIZE>(R[0]);
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
