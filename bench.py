@@ -381,26 +381,13 @@ def build_descs(specs, lay: Layout, x_base: int, y_base: int, s_base: int, idx=N
 
 
 def count_launches(arr) -> int:
-    """Kernel launches of one fp8bq_quantize_batched call over `arr`, grouped the
-    way the library groups tensors: by kernel path and input dtype; then by
-    block shape and, for the vector kernel, by 16-byte or 8-byte-halves row
-    alignment; generic blocks by size class (one CTA per block from 2048
-    elements).  A group launches once per pack of 128 (TMA) or 320 tensors."""
+    """Kernel launches of one fp8bq_quantize_batched call over `arr`, as the
+    library plans them (fp8bq_launch_count)."""
     import blockwise_fp8_weight_b200 as fq
-    groups: dict = {}
-    for d in arr:
-        p = fq.fp8bq_path_for(d)
-        if p == fq.FP8BQ_PATH_GENERIC:
-            key = (p, d.dtype_in, d.block_m * d.block_n >= 2048)
-        else:
-            es = 2 if d.dtype_in == fq.FP8BQ_BF16 else 4
-            vec = 16 // es
-            a16 = (d.x % 16 == 0 and d.ld * es % 16 == 0 and d.N % vec == 0 and d.y_u8 % vec == 0
-                   and (d.batch == 1 or (d.x_batch_stride * es % 16 == 0
-                                         and d.y_batch_stride % vec == 0)))
-            key = (p, d.dtype_in, d.block_m, d.block_n, p == fq.FP8BQ_PATH_VECTOR and not a16)
-        groups[key] = groups.get(key, 0) + 1
-    return sum(-(-n // (128 if k[0] == fq.FP8BQ_PATH_TMA else 320)) for k, n in groups.items())
+    n = fq.fp8bq_launch_count(arr, len(arr))
+    if n < 0:
+        raise RuntimeError("the library rejects this call")
+    return n
 
 
 def cpu_baseline(specs, host: np.ndarray, lay: Layout, seconds: float) -> dict:

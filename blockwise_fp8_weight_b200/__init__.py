@@ -138,6 +138,8 @@ def lib() -> ctypes.CDLL:
             L.fp8bq_get_pdl.restype = i32
             L.fp8bq_path_for.argtypes = [ctypes.POINTER(fp8bq_desc)]
             L.fp8bq_path_for.restype = i32
+            L.fp8bq_launch_count.argtypes = [ctypes.POINTER(fp8bq_desc), i32]
+            L.fp8bq_launch_count.restype = i32
             L.fp8bq_debug_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.fp8bq_debug_set_wait_limit_ns.restype = i32
             L.fp8bq_debug_set_inject.argtypes = [ctypes.c_uint32]
@@ -240,6 +242,15 @@ def fp8bq_get_pdl() -> int:
 
 def fp8bq_path_for(desc: fp8bq_desc) -> int:
     return lib().fp8bq_path_for(ctypes.byref(desc))
+
+
+def fp8bq_launch_count(desc_table, n_tensors=None) -> int:
+    """``fp8bq_launch_count`` of the C ABI: kernel launches the grouped call
+    would enqueue (-1 if it would fail)."""
+    if not isinstance(desc_table, ctypes.Array):
+        desc_table = (fp8bq_desc * len(desc_table))(*desc_table)
+    n = len(desc_table) if n_tensors is None else n_tensors
+    return lib().fp8bq_launch_count(desc_table, n)
 
 
 def fp8bq_debug_set_wait_limit_ns(ns: int) -> int:

@@ -204,6 +204,14 @@ bool tma_geom(const fp8bq_desc &D, int *group, bool *subwarp) {
 // otherwise.
 constexpr int64_t kTmaMinSlotBytes = 16384;
 
+// A call whose TMA tensors hold less input than this runs them on the vector
+// kernel instead.  Measured on B200, one bf16 tensor with 128x128 blocks per
+// call (TMA / vector): 4096x4096 (33 MB of input) 0.783 / 0.848 of the copy
+// peak, 4096x12288 and 12345x4096 (101 MB) 0.890-0.893 / 0.954-0.961,
+// 24576x4096 (201 MB) 0.946 / 0.915, 49152x4096 (403 MB) 0.978 / 0.865; one
+// Qwen3-8B-shaped layer (7 tensors, 386 MB) 0.987 / 0.879.
+constexpr uint64_t kTmaMinCallBytes = 128ull << 20;
+
 Variant choose(const fp8bq_desc &D, int path) {
     if (path == FP8BQ_PATH_GENERIC) return Variant::Generic;
     int g;
@@ -504,7 +512,17 @@ struct GroupKey {
     }
 };
 
-fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
+// The launches of one call: its tensors grouped by kernel variant (the
+// caller's order kept inside a group), with the TMA groups' tensor maps.
+struct Plan {
+    std::vector<GroupKey> keys;
+    std::vector<std::vector<int>> members;
+    std::vector<std::vector<CUtensorMap>> maps;
+};
+
+// Check every descriptor, then group them.  FP8BQ_OK with an empty plan when
+// there is nothing to do.
+fp8bq_status make_plan(const fp8bq_desc *table, int n, Plan &plan) {
     if (n < 0) return FP8BQ_ERR_ARG;
     if (n > 0 && table == nullptr) return FP8BQ_ERR_NULL;
     std::vector<char> empty((size_t)n, 0);
@@ -522,17 +540,32 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
     const fp8bq_status sd = check_device();
     if (sd != FP8BQ_OK) return sd;
 
-    // Group tensors by kernel variant, keeping the caller's order inside a group.
+    // The kernel variant of each tensor.  AUTO sends a call's TMA tensors to
+    // the vector kernel when together they hold less than kTmaMinCallBytes of
+    // input: short launches start sooner on the vector kernel's two CTAs per
+    // SM than on the TMA ring of one CTA per SM.
     const int path = g_path.load();
-    std::vector<GroupKey> keys;
-    std::vector<std::vector<int>> members;
-    std::vector<std::vector<CUtensorMap>> maps;
+    std::vector<Variant> var((size_t)n, Variant::Generic);
+    uint64_t tma_bytes = 0;
     for (int i = 0; i < n; ++i) {
         if (empty[i]) continue;
         const fp8bq_desc &D = table[i];
-        Variant v = choose(D, path);
+        var[i] = choose(D, path);
+        if (var[i] == Variant::Tma)
+            tma_bytes += (uint64_t)D.batch * (uint64_t)D.M * (uint64_t)D.N * esize_of(D.dtype_in);
+    }
+    const bool small_call = path == FP8BQ_PATH_AUTO && tma_bytes < kTmaMinCallBytes;
+
+    std::vector<GroupKey> &keys = plan.keys;
+    std::vector<std::vector<int>> &members = plan.members;
+    std::vector<std::vector<CUtensorMap>> &maps = plan.maps;
+    for (int i = 0; i < n; ++i) {
+        if (empty[i]) continue;
+        const fp8bq_desc &D = table[i];
+        Variant v = var[i];
         CUtensorMap m;
-        if (v == Variant::Tma && !encode_map(D, &m)) v = choose(D, FP8BQ_PATH_VECTOR);
+        if (v == Variant::Tma && (small_call || !encode_map(D, &m)))
+            v = choose(D, FP8BQ_PATH_VECTOR);
         // vector / TMA launches need one block shape; generic ones only one
         // size class (CTA per block for >= 2048 elements, else warp per block)
         const bool big = (int64_t)D.block_m * D.block_n >= 2048;
@@ -549,6 +582,52 @@ fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
         members[g].push_back(i);
         if (v == Variant::Tma) maps[g].push_back(m);
     }
+    return FP8BQ_OK;
+}
+
+// Launches of one group: packs of at most MAXD descriptors and fewer than
+// 2^31 tiles (the chunking of launch_group / launch_tma_group).
+template <int MAXD>
+int packs_of(const fp8bq_desc *t, const std::vector<int> &idx, Variant v) {
+    int packs = 0;
+    size_t i = 0;
+    while (i < idx.size()) {
+        ++packs;
+        int nd = 0;
+        uint64_t total = 0;
+        while (i < idx.size() && nd < MAXD) {
+            const uint64_t tiles = tiles_of(t[idx[i]], v);
+            if (nd > 0 && total + tiles >= (1ull << 31)) break;
+            total += tiles;
+            ++nd;
+            ++i;
+        }
+    }
+    return packs;
+}
+
+int launches_of(const fp8bq_desc *table, const Plan &plan) {
+    int total = 0;
+    for (size_t g = 0; g < plan.keys.size(); ++g) {
+        const std::vector<int> &idx = plan.members[g];
+        const bool small = idx.size() <= (size_t)kMaxDescSmall;
+        const Variant v = plan.keys[g].v;
+        if (v == Variant::Tma)
+            total += small ? packs_of<kMaxDescSmall>(table, idx, v) : packs_of<kMaxDescTma>(table, idx, v);
+        else
+            total += small ? packs_of<kMaxDescSmall>(table, idx, v)
+                           : packs_of<kMaxDescLarge>(table, idx, v);
+    }
+    return total;
+}
+
+fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
+    Plan plan;
+    const fp8bq_status sp = make_plan(table, n, plan);
+    if (sp != FP8BQ_OK || plan.keys.empty()) return sp;
+    const std::vector<GroupKey> &keys = plan.keys;
+    const std::vector<std::vector<int>> &members = plan.members;
+    const std::vector<std::vector<CUtensorMap>> &maps = plan.maps;
     auto launch = [&](size_t g, cudaStream_t st) -> cudaError_t {
         if (keys[g].v == Variant::Tma)
             return members[g].size() <= (size_t)kMaxDescSmall
@@ -883,6 +962,12 @@ int fp8bq_path_for(const fp8bq_desc *desc) {
         case Variant::Generic: return FP8BQ_PATH_GENERIC;
         default: return FP8BQ_PATH_VECTOR;
     }
+}
+
+int fp8bq_launch_count(const fp8bq_desc *desc_table, int n_tensors) {
+    Plan plan;
+    if (make_plan(desc_table, n_tensors, plan) != FP8BQ_OK) return -1;
+    return launches_of(desc_table, plan);
 }
 
 fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns) {

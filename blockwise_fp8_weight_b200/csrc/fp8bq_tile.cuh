@@ -122,15 +122,17 @@ struct TileCursor {
     }
 };
 
-// absmax bits of one 16-byte vector: a tree of three maxima.
+// absmax bits of one 16-byte vector: a tree of three maxima (the integer
+// form needs sign-cleared first operands; the xorsign form ignores signs).
 template <int ESIZE>
 __device__ __forceinline__ uint32_t vec_absmax(const uint4 &v) {
+    constexpr uint32_t keep = FP8BQ_ABSMAX_FMAX ? 0xffffffffu : ESIZE == 2 ? 0x7fff7fffu
+                                                                          : 0x7fffffffu;
     if constexpr (ESIZE == 2)
-        return dev::absmax_bf16x2(dev::absmax_bf16x2(v.x & 0x7fff7fffu, v.y),
-                                  dev::absmax_bf16x2(v.z & 0x7fff7fffu, v.w));
+        return dev::absmax_bf16x2(dev::absmax_bf16x2(v.x & keep, v.y),
+                                  dev::absmax_bf16x2(v.z & keep, v.w));
     else
-        return dev::absmax_f32(dev::absmax_f32(v.x & 0x7fffffffu, v.y),
-                               dev::absmax_f32(v.z & 0x7fffffffu, v.w));
+        return dev::absmax_f32(dev::absmax_f32(v.x & keep, v.y), dev::absmax_f32(v.z & keep, v.w));
 }
 
 // absmax bits of V 16-byte vectors: four independent running maxima (one per

@@ -272,9 +272,20 @@ FP8BQ_API fp8bq_path fp8bq_get_path(void);
 /*
  * Which variant a tensor would take under the current selection (host only,
  * launches nothing).  Returns FP8BQ_PATH_VECTOR, _TMA or _GENERIC, or -1 if
- * the descriptor is invalid.
+ * the descriptor is invalid.  This is the tensor's own choice; under AUTO a
+ * call whose TMA tensors hold less than 128 MiB of input in all runs them on
+ * the vector kernel (short launches start sooner there), which
+ * fp8bq_launch_count accounts for.
  */
 FP8BQ_API int fp8bq_path_for(const fp8bq_desc *desc);
+
+/*
+ * Number of kernel launches fp8bq_quantize_batched(desc_table, n_tensors, .)
+ * would enqueue under the current selection (host only, launches nothing;
+ * needs a usable device, like the call itself).  Returns -1 if the call would
+ * return an error.
+ */
+FP8BQ_API int fp8bq_launch_count(const fp8bq_desc *desc_table, int n_tensors);
 
 /*
  * Programmatic dependent launch (process-wide; on by default).  When on,

@@ -26,7 +26,7 @@ int main(void) {
         (fn)fp8bq_sync_status,    (fn)fp8bq_version,          (fn)fp8bq_set_path,
         (fn)fp8bq_get_path,       (fn)fp8bq_path_for,         (fn)fp8bq_set_pdl,
         (fn)fp8bq_get_pdl,        (fn)fp8bq_debug_set_wait_limit_ns,
-        (fn)fp8bq_debug_set_inject,
+        (fn)fp8bq_debug_set_inject, (fn)fp8bq_launch_count,
     };
     size_t i;
     for (i = 0; i < sizeof entry / sizeof entry[0]; ++i) CHECK(entry[i] != NULL);
@@ -47,6 +47,7 @@ int main(void) {
         CHECK(fp8bq_quantize((const void *)0x1000, FP8BQ_BF16, 4, 8, 7, 128, 128, y, s, 0) ==
               FP8BQ_ERR_SHAPE);
         CHECK(fp8bq_quantize_batched(NULL, -1, 0) == FP8BQ_ERR_ARG);
+        CHECK(fp8bq_launch_count(NULL, -1) == -1);
         CHECK(fp8bq_quantize_batched(NULL, 0, 0) == FP8BQ_OK); /* nothing to do */
     }
 

@@ -142,6 +142,15 @@ def path_guard():
     fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
 
 
+def test_launch_count_refuses_what_the_call_refuses():
+    assert fq.fp8bq_launch_count([desc(block_m=0)]) == -1        # invalid block
+    assert fq.fp8bq_launch_count([desc()], n_tensors=-1) == -1   # negative count
+    # a valid call needs a usable device to be planned (none in this container
+    # means -1; on a B200 the GPU tests check the counts)
+    if not torch.cuda.is_available():
+        assert fq.fp8bq_launch_count([desc()]) == -1
+
+
 def test_variant_choice(path_guard):
     P = fq.fp8bq_path_for
     assert fq.fp8bq_get_path() == fq.FP8BQ_PATH_AUTO

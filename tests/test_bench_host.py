@@ -104,23 +104,13 @@ def test_reference_arm_other_ranks_exit_quietly():
     assert out.returncode == 0 and out.stdout.strip() == ""
 
 
-def test_shape_workload_and_launch_count():
-    """`shape:` builds one tensor of the given shape; the launch count mirrors
-    the library's grouping (dtype, block shape, 16-byte or 8-byte-halves row
-    alignment, generic size class) without a GPU."""
+def test_shape_workload():
+    """`shape:` builds one tensor of the given shape (the launch counts the
+    bench reports come from the library's own plan, checked on the GPU)."""
     (sp,), _ = bench.workload("shape:128x1536x2048")
     assert (sp.batch, sp.M, sp.N, sp.dtype) == (128, 1536, 2048, "bf16")
     (sp,), _ = bench.workload("shape:4000x4100:f32")
     assert (sp.batch, sp.M, sp.N, sp.dtype) == (1, 4000, 4100, "f32")
-    specs, _ = bench.workload("edge")
-    lay = bench.Layout(specs)
-    table = bench.build_descs(specs, lay, 1 << 40, 1 << 41, 1 << 42)
-    # bf16: TMA, vector halves (4000x4100 and its ld=4164 twin), vector 1x128,
-    # vector 64x64, generic; fp32: TMA, generic
-    assert bench.count_launches(table) == 7
-    qwen = W.qwen3_8b_model()
-    lay = bench.Layout(qwen)
-    assert bench.count_launches(bench.build_descs(qwen, lay, 1 << 40, 1 << 41, 1 << 42)) == 2
 
 
 def test_traffic_record_lookup(tmp_path, monkeypatch):

@@ -375,3 +375,43 @@ def test_mixed_variant_call_in_a_cuda_graph(edge_case):
     assert fq.fp8bq_sync_status() == fq.FP8BQ_OK
     for sp, o, w in zip(case.specs, outs, case.want):
         assert_same(sp, o.result(), w)
+
+
+def test_launch_count_follows_the_plan(qwen_layer_case):
+    """fp8bq_launch_count reports the launches of a call as planned: one per
+    kernel variant, dtype and block shape and per pack of descriptors (128 for
+    the TMA kernel, 320 for the others), with AUTO's per-call size rule (a
+    call whose TMA tensors hold less than 128 MiB of input runs them on the
+    vector kernel)."""
+    from tests.gpu_util import Outputs
+    lay = [Outputs(sp).desc(p) for sp, p in zip(qwen_layer_case.specs, qwen_layer_case.ptrs)]
+    assert fq.fp8bq_launch_count(lay) == 1                     # 386 MB: one TMA launch
+    one = lay[1]                                               # k_proj alone: 8 MB
+    assert fq.fp8bq_path_for(one) == fq.FP8BQ_PATH_TMA        # its own choice ...
+    assert fq.fp8bq_launch_count([one]) == 1                   # ... one (vector) launch
+    sp = TensorSpec("count", 256, 256, seed=1)
+    owner, ptr = to_device(W.materialize(sp))
+    many = [Outputs(sp) for _ in range(200)]                  # 200 small tensors, 26 MB
+    descs = [o.desc(ptr) for o in many]
+    assert fq.fp8bq_launch_count(descs) == 1                   # one vector pack of <= 320
+    assert fq.fp8bq_set_path(fq.FP8BQ_PATH_TMA) == fq.FP8BQ_OK
+    try:
+        assert fq.fp8bq_launch_count(descs) == 2               # TMA packs of <= 128
+        assert fq.fp8bq_launch_count(descs + [lay[0]]) == 2    # q_proj joins the second pack
+    finally:
+        fq.fp8bq_set_path(fq.FP8BQ_PATH_AUTO)
+    del owner
+
+
+def test_bench_launch_counts():
+    """The launch counts the benchmark reports (from the library's plan): the
+    edge set takes 7 launches (bf16: TMA pairs, vector halves, vector 1x128,
+    vector 64x64, generic; fp32: TMA, generic), the whole weight set 2 (TMA
+    packs of 128 and 124 tensors)."""
+    import bench
+    specs, _ = bench.workload("edge")
+    lay = bench.Layout(specs)
+    assert bench.count_launches(bench.build_descs(specs, lay, 1 << 40, 1 << 41, 1 << 42)) == 7
+    qwen = W.qwen3_8b_model()
+    lay = bench.Layout(qwen)
+    assert bench.count_launches(bench.build_descs(qwen, lay, 1 << 40, 1 << 41, 1 << 42)) == 2
