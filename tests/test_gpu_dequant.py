@@ -76,16 +76,20 @@ CASES = [
     TensorSpec("b64", 200, 192, block=(64, 64), seed=81, tensor_id=5),
     TensorSpec("experts", 256, 768, batch=4, seed=81, tensor_id=6, batch_lognormal_sigma=0.7),
     TensorSpec("odd_block", 100, 96, block=(5, 48), seed=81, tensor_id=7),
+    TensorSpec("tile_edges", 130, 400, block=(32, 16), seed=81, tensor_id=8),  # ragged tiles
 ]
 
 
 @pytest.mark.parametrize("sp", CASES, ids=[c.name for c in CASES])
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("path", ["auto", "generic"])
+@pytest.mark.parametrize("path", ["auto", "vector", "generic"])
 def test_dequantize_matches_oracle(sp, out_dtype, path):
+    """AUTO takes the TMA-store kernel where it can (power-of-two blocks,
+    16-byte aligned rows), VECTOR forces the register kernel."""
     y, s = quantized(sp)
     want = expected(y, s, *sp.block, out_dtype)
-    P = fq.FP8BQ_PATH_AUTO if path == "auto" else fq.FP8BQ_PATH_GENERIC
+    P = {"auto": fq.FP8BQ_PATH_AUTO, "vector": fq.FP8BQ_PATH_VECTOR,
+         "generic": fq.FP8BQ_PATH_GENERIC}[path]
     got = run_dequant(y, s, sp.M, sp.N, *sp.block, out_dtype, batch=sp.batch, path=P)
     assert np.array_equal(got.view(np.uint32 if out_dtype == "f32" else np.uint16),
                           want.view(np.uint32 if out_dtype == "f32" else np.uint16))

@@ -384,7 +384,8 @@ def test_launch_count_follows_the_plan(qwen_layer_case):
     call whose TMA tensors hold less than 128 MiB of input runs them on the
     vector kernel)."""
     from tests.gpu_util import Outputs
-    lay = [Outputs(sp).desc(p) for sp, p in zip(qwen_layer_case.specs, qwen_layer_case.ptrs)]
+    outs = [Outputs(sp) for sp in qwen_layer_case.specs]      # kept alive: distinct outputs
+    lay = [o.desc(p) for o, p in zip(outs, qwen_layer_case.ptrs)]
     assert fq.fp8bq_launch_count(lay) == 1                     # 386 MB: one TMA launch
     one = lay[1]                                               # k_proj alone: 8 MB
     assert fq.fp8bq_path_for(one) == fq.FP8BQ_PATH_TMA        # its own choice ...
