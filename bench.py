@@ -700,6 +700,7 @@ def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_de
     nbytes = sum(sp.numel * 3 + sp.nblocks * 4 for sp in specs)
     value = aggregate(nbytes, args.steps, world, el)
     peak, kind = measured_peak()
+    dq_launches = -(-len(specs) // 320)  # 320 descriptors per launch
     if rank == 0:
         print(json.dumps({
             "metric": "blockwise FP8 dequantize GB/s (e4m3 codes + descales in, bf16 out)",
@@ -709,11 +710,11 @@ def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_de
             "data": "synthetic",
             "config": {"workload": wl_desc + " (dequantize its codes to bf16)",
                        "name": args.workload, "op": "dequantize", "bytes_per_step": nbytes,
-                       "launches_per_step": -(-len(specs) // 320)},
+                       "launches_per_step": dq_launches, "path": args.path},
             "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
                          "frac": value / world / peak, "traffic": None,
                          "peak_source": kind},
-            "gpu_launches": -(-len(specs) // 320) * args.steps, "clocks": clk.summary()}),
+            "gpu_launches": dq_launches * args.steps, "clocks": clk.summary()}),
               flush=True)
 
 

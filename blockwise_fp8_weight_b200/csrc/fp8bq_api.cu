@@ -711,101 +711,6 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
     return cudaSuccess;
 }
 
-// The TMA dequantization kernel takes what the vector one takes, with block
-// shapes that are powers of two; its output is a tensor map (16-byte aligned
-// base and strides, which the vector conditions already require).
-bool dequant_tma_ok(const fp8bq_dequant_desc &D) {
-    const uint64_t tiles = (uint64_t)D.batch * (uint64_t)cdiv(D.M, kDqTileRows) *
-                           (uint64_t)cdiv(D.N, kDqTileCols);
-    return dequant_vector_ok(D) && is_pow2(D.block_m) && is_pow2(D.block_n) &&
-           tiles < (1ull << 31);
-}
-
-// The output of a dequantization as a 3-D tensor map {N, M, batch}, box
-// {kDqTileCols, kDqTileRows, 1}, cached like the input maps.
-bool encode_out_map(const fp8bq_dequant_desc &D, CUtensorMap *out) {
-    static std::mutex mu;
-    static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
-    MapKey key;
-    std::memset(&key, 0, sizeof key);
-    key.x = (uintptr_t)D.out;
-    key.M = D.M;
-    key.N = D.N;
-    key.ld = D.ld_out;
-    key.batch = D.batch;
-    key.xbs = D.batch > 1 ? D.out_batch_stride : D.M * D.ld_out;
-    key.dtype = D.dtype_out;
-    {
-        std::lock_guard<std::mutex> g(mu);
-        auto it = cache.find(key);
-        if (it != cache.end()) {
-            *out = it->second;
-            return true;
-        }
-    }
-    auto fn = encode_fn();
-    if (!fn) return false;
-    const int es = esize_of(D.dtype_out);
-    cuuint64_t dims[3] = {(cuuint64_t)D.N, (cuuint64_t)D.M, (cuuint64_t)D.batch};
-    cuuint64_t strides[2] = {(cuuint64_t)(D.ld_out * es), (cuuint64_t)(key.xbs * es)};
-    cuuint32_t box[3] = {(cuuint32_t)kDqTileCols, (cuuint32_t)kDqTileRows, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUtensorMap m;
-    CUresult r = fn(&m,
-                    D.dtype_out == FP8BQ_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                              : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                    3, D.out, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return false;
-    std::lock_guard<std::mutex> g(mu);
-    if (cache.size() > 8192) cache.clear();
-    cache.emplace(key, m);
-    *out = m;
-    return true;
-}
-
-template <int MAXD>
-cudaError_t launch_dequant_tma_group(const fp8bq_dequant_desc *t, const std::vector<int> &idx,
-                                     const std::vector<CUtensorMap> &maps, int oes,
-                                     cudaStream_t st) {
-    static thread_local DequantTmaPack<MAXD> P;
-    size_t i = 0;
-    while (i < idx.size()) {
-        DequantPack<MAXD> &p = P.p;
-        p.n = 0;
-        p.pad_ = 0;
-        p.total = 0;
-        while (i < idx.size() && p.n < MAXD) {
-            const fp8bq_dequant_desc &D = t[idx[i]];
-            DequantDesc &o = p.d[p.n];
-            o.y = D.y_u8;
-            o.s = D.descale_f32;
-            o.out = D.out;
-            o.M = D.M;
-            o.N = D.N;
-            o.ldo = D.ld_out;
-            o.obs = D.batch > 1 ? D.out_batch_stride : 0;
-            o.bm = D.block_m;
-            o.bn = D.block_n;
-            o.gm = (int32_t)cdiv(D.M, D.block_m);
-            o.gn = (int32_t)cdiv(D.N, D.block_n);
-            o.bm_log2 = __builtin_ctz((unsigned)D.block_m);
-            o.bn_log2 = __builtin_ctz((unsigned)D.block_n);
-            o.begin = p.total;
-            o.items = (uint64_t)D.batch * (uint64_t)cdiv(D.M, kDqTileRows) *
-                      (uint64_t)cdiv(D.N, kDqTileCols);
-            P.maps[p.n] = maps[i];
-            p.total += o.items;
-            ++p.n;
-            ++i;
-        }
-        const cudaError_t e = launch_dequant_tma<MAXD>(P, oes, st);
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
-}
-
 fp8bq_status run_dequant(const fp8bq_dequant_desc *t, int n, cudaStream_t stream) {
     if (n < 0) return FP8BQ_ERR_ARG;
     if (n > 0 && t == nullptr) return FP8BQ_ERR_NULL;
@@ -845,33 +750,20 @@ fp8bq_status run_dequant(const fp8bq_dequant_desc *t, int n, cudaStream_t stream
     }
     const fp8bq_status sd = check_device();
     if (sd != FP8BQ_OK) return sd;
-    // kind 0: generic, 1: vector, 2: TMA (AUTO and TMA selections)
-    const int path = g_path.load();
-    std::vector<int> groups[3][2];  // [kind][output is bf16]
-    std::vector<CUtensorMap> maps[2];  // of the TMA groups, [output is bf16]
+    const bool generic_only = g_path.load() == FP8BQ_PATH_GENERIC;
+    std::vector<int> groups[2][2];  // [vector][output is bf16]
     for (int i = 0; i < n; ++i) {
         if (empty[i]) continue;
-        const bool bf = t[i].dtype_out == FP8BQ_BF16;
-        int kind = path != FP8BQ_PATH_GENERIC && dequant_vector_ok(t[i]) ? 1 : 0;
-        CUtensorMap m;
-        if (kind == 1 && path != FP8BQ_PATH_VECTOR && dequant_tma_ok(t[i]) &&
-            encode_out_map(t[i], &m)) {
-            kind = 2;
-            maps[bf].push_back(m);
-        }
-        groups[kind][bf].push_back(i);
+        const bool v = !generic_only && dequant_vector_ok(t[i]);
+        groups[v][t[i].dtype_out == FP8BQ_BF16].push_back(i);
     }
-    std::vector<std::pair<int, int>> used;  // (kind, bf16 output) of each non-empty group
-    for (int v = 0; v < 3; ++v)
+    std::vector<std::pair<int, int>> used;  // (vector, bf16 output) of each non-empty group
+    for (int v = 0; v < 2; ++v)
         for (int b = 0; b < 2; ++b)
             if (!groups[v][b].empty()) used.emplace_back(v, b);
     auto launch = [&](size_t k, cudaStream_t st) -> cudaError_t {
         const int v = used[k].first, b = used[k].second;
         const std::vector<int> &g = groups[v][b];
-        if (v == 2)
-            return g.size() <= (size_t)kMaxDescSmall
-                       ? launch_dequant_tma_group<kMaxDescSmall>(t, g, maps[b], b ? 2 : 4, st)
-                       : launch_dequant_tma_group<kMaxDescTma>(t, g, maps[b], b ? 2 : 4, st);
         return g.size() <= (size_t)kMaxDescSmall
                    ? launch_dequant_group<kMaxDescSmall>(t, g, v, b ? 2 : 4, st)
                    : launch_dequant_group<kMaxDescLarge>(t, g, v, b ? 2 : 4, st);

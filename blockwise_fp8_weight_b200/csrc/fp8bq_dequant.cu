@@ -8,7 +8,8 @@
 //
 // decode() is exact in two steps: cvt.rn.f16x2.e4m3x2 (every e4m3fn value,
 // subnormals included, is a normal fp16 value) and fp16 -> fp32.
-#include "fp8bq_tile.cuh"
+#include "fp8bq_device.cuh"
+#include "fp8bq_internal.h"
 
 namespace fp8bq {
 namespace {
@@ -56,7 +57,11 @@ __device__ __forceinline__ const DequantDesc &find(const DequantPack<MAXD> &p, u
 #define FP8BQ_DQ_UNROLL 2  // measured: 1 -> 4.36, 2 -> 5.41, 4 -> 5.61 TB/s on one layer,
                            // 4.64 / 5.58 / 5.48 TB/s on the whole weight set
 #endif
-// Measured and dropped: numbering the items in 32 bits with shifts for
+// Measured and dropped: 64 x 128 output tiles written into shared memory and
+// handed to TMA tile stores (72.9 M instructions on one layer, about the
+// same as here, and 121 us instead of 108 us cold; 0.69-0.72 of the copy
+// peak live against 0.84: two CTA barriers per tile and one issuing thread
+// serialise the tiles); numbering the items in 32 bits with shifts for
 // power-of-two blocks (43.9 M instead of 75.2 M instructions on one layer,
 // yet 142 us instead of 108 us: with the index arithmetic gone, nothing
 // hides the load latency -- long-scoreboard stalls 21 per issue against
@@ -158,118 +163,6 @@ __global__ void __launch_bounds__(256)
     }
 }
 
-// TMA kernel: a CTA of 256 threads per output tile of 64 x 128 elements.
-// Thread t holds the 8 codes (row t / 16 + 16 s, column 8 (t % 16)) of the
-// tile for s < 4 -- 8-byte loads, the next tile's issued before the current
-// one is processed -- and writes their 8 outputs as one 16-byte shared
-// store (consecutive threads, consecutive 16 bytes: no bank conflicts) into
-// one of two tile buffers; after a barrier one thread hands the tile to the
-// TMA, which writes it to the output (elements beyond M or N are not
-// written) while the CTA goes on with the next tile in the other buffer.
-// Block shapes are powers of two (the descale of a chunk takes two shifts).
-template <int OES, int MAXD>
-__global__ void __launch_bounds__(256) k_dequant_tma(const __grid_constant__ DequantTmaPack<MAXD> P) {
-    dev::pdl_entry();
-    constexpr int TR = kDqTileRows, TC = kDqTileCols, STEPS = TR * TC / (256 * 8);
-    constexpr int BUF = TR * TC * OES;  // one output tile
-    extern __shared__ __align__(1024) uint8_t obuf[];
-    const DequantPack<MAXD> &p = P.p;
-    const int tid = threadIdx.x;
-    const int rl = tid >> 4, cl = (tid & 15) * 8;
-    int d = 0;
-
-    struct Pos {
-        int d;
-        uint32_t b, r0, c0;
-    };
-    auto locate = [&](uint64_t t) -> Pos {
-        const DequantDesc &a = find(p, t, d);
-        const uint32_t local = (uint32_t)(t - a.begin);
-        const uint32_t tcn = (uint32_t)((a.N + TC - 1) / TC);
-        const uint32_t per = (uint32_t)((a.M + TR - 1) / TR) * tcn;
-        const uint32_t b = local / per;
-        const uint32_t rem = local - b * per;
-        const uint32_t tr = rem / tcn;
-        return Pos{d, b, tr * TR, (rem - tr * tcn) * TC};
-    };
-    auto load = [&](const Pos &q, uint2 (&c)[STEPS]) {
-        const DequantDesc &a = p.d[q.d];
-        const int64_t col = (int64_t)q.c0 + cl;
-        const uint8_t *base = a.y + ((int64_t)q.b * a.M) * a.N + col;
-#pragma unroll
-        for (int s = 0; s < STEPS; ++s) {
-            const int64_t r = (int64_t)q.r0 + rl + 16 * s;
-            if (r < a.M && col < a.N)  // N is a multiple of 16: the 8 codes are all inside
-                c[s] = dev::ldg_v2(base + r * a.N);
-            else
-                c[s] = make_uint2(0u, 0u);
-        }
-    };
-
-    uint64_t t = blockIdx.x;
-    if (t >= p.total) return;
-    Pos cur = locate(t);
-    uint2 qc[STEPS];
-    load(cur, qc);
-    for (uint32_t k = 0;; ++k) {
-        const uint64_t tn = t + gridDim.x;
-        const bool more = tn < p.total;
-        Pos nxt = cur;
-        uint2 qn[STEPS];
-        if (more) {
-            nxt = locate(tn);
-            load(nxt, qn);  // in flight while this tile is processed
-        }
-        uint8_t *buf = obuf + (k & 1) * BUF;
-        if (tid == 0 && k >= 2) dev::bulk_wait_group_read<1>();  // this buffer's last store read it
-        __syncthreads();
-        const DequantDesc &a = p.d[cur.d];
-        const int64_t col = (int64_t)cur.c0 + cl;
-        const float *srow = a.s + (int64_t)cur.b * a.gm * a.gn + (col >> a.bn_log2);
-#pragma unroll
-        for (int s = 0; s < STEPS; ++s) {
-            // outside the matrix: no descale read (the TMA store drops these)
-            const int64_t r = (int64_t)cur.r0 + rl + 16 * s;
-            const float sc = r < a.M && col < a.N ? __ldg(srow + (r >> a.bm_log2) * a.gn) : 0.0f;
-            uint64_t ss;
-            asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(sc));
-            float v[8];
-            decode2((uint16_t)(qc[s].x & 0xffffu), v[0], v[1]);
-            decode2((uint16_t)(qc[s].x >> 16), v[2], v[3]);
-            decode2((uint16_t)(qc[s].y & 0xffffu), v[4], v[5]);
-            decode2((uint16_t)(qc[s].y >> 16), v[6], v[7]);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
-            uint8_t *o = buf + ((rl + 16 * s) * TC + cl) * OES;
-            if constexpr (OES == 2) {
-                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dev::smem_addr(o)),
-                             "r"(pack_bf16x2(v[0], v[1])), "r"(pack_bf16x2(v[2], v[3])),
-                             "r"(pack_bf16x2(v[4], v[5])), "r"(pack_bf16x2(v[6], v[7]))
-                             : "memory");
-            } else {
-                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dev::smem_addr(o)),
-                             "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3])
-                             : "memory");
-                asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dev::smem_addr(o + 16)),
-                             "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7])
-                             : "memory");
-            }
-        }
-        dev::fence_proxy_async_shared();  // the stores above, visible to the TMA
-        __syncthreads();
-        if (tid == 0) {
-            dev::tma_store_3d(&P.maps[cur.d], buf, (int)cur.c0, (int)cur.r0, (int)cur.b);
-            dev::bulk_commit_group();
-        }
-        if (!more) break;
-        t = tn;
-        cur = nxt;
-#pragma unroll
-        for (int s = 0; s < STEPS; ++s) qc[s] = qn[s];
-    }
-    if (tid == 0) dev::bulk_wait_group_all();  // every tile written before the CTA exits
-}
-
 unsigned dq_grid(uint64_t work) {
     const uint64_t need = (work + 255) / 256;
     const uint64_t cap = (uint64_t)sm_count() * 8;
@@ -290,25 +183,6 @@ cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vecto
                           : launch_kernel(k_dequant_generic<4, MAXD>, grid, 256, 0, st, p);
 }
 
-template <int MAXD>
-cudaError_t launch_dequant_tma(const DequantTmaPack<MAXD> &p, int out_esize, cudaStream_t st) {
-    auto go = [&](auto kern, size_t smem, PerDevice<KernelSetup> &setup) {
-        const KernelSetup ks = setup.get([&] { return setup_kernel(kern, 256, smem); });
-        if (ks.attr != cudaSuccess) return ks.attr;
-        const uint64_t cap = (uint64_t)sm_count() * (uint64_t)ks.occ;
-        const unsigned grid = (unsigned)(p.p.total < cap ? p.p.total : cap);
-        return launch_kernel(kern, grid, 256, smem, st, p);
-    };
-    static PerDevice<KernelSetup> setup2, setup4;
-    return out_esize == 2
-               ? go(k_dequant_tma<2, MAXD>, (size_t)2 * kDqTileRows * kDqTileCols * 2, setup2)
-               : go(k_dequant_tma<4, MAXD>, (size_t)2 * kDqTileRows * kDqTileCols * 4, setup4);
-}
-
-template cudaError_t launch_dequant_tma<kMaxDescSmall>(const DequantTmaPack<kMaxDescSmall> &, int,
-                                                       cudaStream_t);
-template cudaError_t launch_dequant_tma<kMaxDescTma>(const DequantTmaPack<kMaxDescTma> &, int,
-                                                     cudaStream_t);
 template cudaError_t launch_dequant<kMaxDescSmall>(const DequantPack<kMaxDescSmall> &, int, bool,
                                                    cudaStream_t);
 template cudaError_t launch_dequant<kMaxDescLarge>(const DequantPack<kMaxDescLarge> &, int, bool,

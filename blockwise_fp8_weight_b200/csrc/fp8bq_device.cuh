@@ -273,33 +273,6 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, ui
     }
 }
 
-// 3-D TMA tile store from shared memory (bulk async-group completion);
-// elements outside the tensor map's extents are not written.
-__device__ __forceinline__ void tma_store_3d(const void *tmap, const void *smem_src, int c0, int c1,
-                                             int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-            tmap),
-        "r"(smem_addr(smem_src)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() {
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-// Wait until at most N of this thread's bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_group_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
-}
-// Wait until all of this thread's bulk groups have completed.
-__device__ __forceinline__ void bulk_wait_group_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-// Make this thread's shared-memory writes visible to the TMA (async proxy).
-__device__ __forceinline__ void fence_proxy_async_shared() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // Named barrier over `count` threads.
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

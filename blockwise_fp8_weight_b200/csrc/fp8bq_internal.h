@@ -172,9 +172,8 @@ struct DequantDesc {
     int32_t bm, bn, gm, gn;
     uint64_t begin;     // first work item of this descriptor
     uint64_t items;     // work items of this descriptor
-    int32_t bm_log2, bn_log2;  // log2 of the block shape (TMA kernel: powers of two)
 };
-static_assert(sizeof(DequantDesc) == 96, "DequantDesc layout");
+static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
 
 template <int MAXD>
 struct DequantPack {
@@ -187,20 +186,6 @@ static_assert(sizeof(DequantPack<kMaxDescLarge>) < 32000, "kernel parameter limi
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st);
-
-// TMA dequantization: work items are output tiles of kDqTileRows x
-// kDqTileCols elements of one matrix; each is written back by one TMA tile
-// store from shared memory (maps[d]: the output of descriptor d as a 3-D
-// tensor {N, M, batch}, box {kDqTileCols, kDqTileRows, 1}).
-constexpr int kDqTileRows = 64, kDqTileCols = 128;
-template <int MAXD>
-struct alignas(64) DequantTmaPack {
-    CUtensorMap maps[MAXD];
-    DequantPack<MAXD> p;
-};
-static_assert(sizeof(DequantTmaPack<kMaxDescTma>) < 32000, "kernel parameter limit");
-template <int MAXD>
-cudaError_t launch_dequant_tma(const DequantTmaPack<MAXD> &p, int out_esize, cudaStream_t st);
 // 16-byte code chunks per lane in a work item of the vector dequant kernel
 int dequant_unroll();
 

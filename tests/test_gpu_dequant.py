@@ -84,8 +84,8 @@ CASES = [
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("path", ["auto", "vector", "generic"])
 def test_dequantize_matches_oracle(sp, out_dtype, path):
-    """AUTO takes the TMA-store kernel where it can (power-of-two blocks,
-    16-byte aligned rows), VECTOR forces the register kernel."""
+    """Every kernel: AUTO (the vector kernel where rows and blocks allow it),
+    VECTOR forced, GENERIC forced."""
     y, s = quantized(sp)
     want = expected(y, s, *sp.block, out_dtype)
     P = {"auto": fq.FP8BQ_PATH_AUTO, "vector": fq.FP8BQ_PATH_VECTOR,
