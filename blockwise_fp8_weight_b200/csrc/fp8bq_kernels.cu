@@ -43,29 +43,27 @@ namespace fp8bq {
 // Reduce-scatter of 8 per-lane maxima over an aligned team of 16 lanes:
 // three halving exchange steps (xor 8, 4, 2) and one full step (xor 1).
 // Afterwards team lane q holds the team-wide max of slot 4*b3 + 2*b2 + b1
-// (b_k = bit k of q), i.e. slot q / 2; 8 shuffles instead of 32.  `merge`
-// combines two running maxima (packed bf16 magnitudes or fp32 ones).
-template <typename Merge>
+// (b_k = bit k of q), i.e. slot q / 2; 8 shuffles instead of 32.
 __device__ __forceinline__ uint32_t reduce_scatter8x16(const uint32_t (&m)[8], uint32_t mask,
-                                                      int q, Merge merge) {
+                                                      int q) {
     const bool h3 = q & 8, h2 = q & 4, h1 = q & 2;
     uint32_t a[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t send = h3 ? m[j] : m[j + 4];
         const uint32_t keep = h3 ? m[j + 4] : m[j];
-        a[j] = merge(keep, __shfl_xor_sync(mask, send, 8));
+        a[j] = max(keep, __shfl_xor_sync(mask, send, 8));
     }
     uint32_t b[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         const uint32_t send = h2 ? a[j] : a[j + 2];
         const uint32_t keep = h2 ? a[j + 2] : a[j];
-        b[j] = merge(keep, __shfl_xor_sync(mask, send, 4));
+        b[j] = max(keep, __shfl_xor_sync(mask, send, 4));
     }
     const uint32_t send = h1 ? b[0] : b[1];
-    uint32_t c = merge(h1 ? b[1] : b[0], __shfl_xor_sync(mask, send, 2));
-    return merge(c, __shfl_xor_sync(mask, c, 1));
+    uint32_t c = max(h1 ? b[1] : b[0], __shfl_xor_sync(mask, send, 2));
+    return max(c, __shfl_xor_sync(mask, c, 1));
 }
 
 // vec_quant_store for a lane's 16 bytes held as two 8-byte halves (rows that
@@ -148,10 +146,9 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     // Every slot of every lane of the team lies inside the tile (the same for
     // the whole team): the interior tiles skip the per-vector bounds checks.
     auto is_full = [&](const Tile &T) { return T.rows >= V * rstep && T.cols >= vpr * VEC; };
-    // Quantize and store slot i of every lane with the reciprocal rr(i): every
-    // slot inside the tile (a slot of a block below the matrix lies below it
-    // too, so the row check covers both).
-    auto store_all = [&](const uint4 (&R)[V], const Tile &T, auto rr_of) {
+    // Quantize and store slot i of every lane for i < nb (the slots of blocks
+    // inside the matrix), with the reciprocal rr(i).
+    auto store_all = [&](const uint4 (&R)[V], const Tile &T, int nb, auto rr_of) {
         uint8_t *dst = T.dst + (int64_t)row0 * T.ldy + colv;
         const int64_t ystep = (int64_t)rstep * T.ldy;
         if (is_full(T)) {
@@ -160,9 +157,11 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         } else {
             const bool hi = hi_ok(T);
 #pragma unroll
-            for (int i = 0; i < V; ++i)
+            for (int i = 0; i < V; ++i) {
+                if (i >= nb) break;
                 if (row0 + i * rstep < T.rows && colv < T.cols)
                     store(R[i], rr_of(i), dst + i * ystep, hi);
+            }
         }
     };
 
@@ -189,23 +188,28 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
       if constexpr (TEAM == 16 && V == 8) {  // the only stacked-block instantiation
         const int bm = p.d[0].bm;
         // each slot's maximum as fp32 bits, then integer maxima through the
-        // reduce-scatter (measured: keeping the maxima packed as bf16 pairs
-        // and merging them with the bf16 max there instead costs 3 % -- it
-        // moves work onto the pipe the conversions already load)
+        // reduce-scatter.  Measured and dropped: keeping the maxima packed as
+        // bf16 pairs merged with the bf16 max there, a three-max absmax per
+        // vector, and no per-tile block count -- 0.87-0.88 of the copy peak
+        // together against 0.90 for this form (same box, A/B); each alone
+        // moved little, the generated code at the 128-register bound did.
         uint32_t m[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) m[i] = absmax_to_f32_bits<ESIZE>(vec_absmax<ESIZE>(R[i]));
+        for (int i = 0; i < V; ++i) {
+            const uint4 one[1] = {R[i]};
+            m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
+        }
         // lane q ends with the max of slot q / 2, computes its scale, and the
         // reciprocal of slot i is fetched from lane 2 i of the team
-        const uint32_t mq = reduce_scatter8x16(m, shfl_mask, lane,
-                                               [](uint32_t a, uint32_t b) { return max(a, b); });
+        const uint32_t mq = reduce_scatter8x16(m, shfl_mask, lane);
         float s_mine, r_mine;
         dev::block_scale(mq, kEps, s_mine, r_mine);
         const int base = (threadIdx.x & 31) & ~(TEAM - 1);
         float r[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + 2 * i);
-        store_all(R, T, [&](int i) { return dev::splat2(r[i]); });
+        // slots of blocks below the matrix are neither quantized nor stored
+        store_all(R, T, (T.rows + bm - 1) / bm, [&](int i) { return dev::splat2(r[i]); });
         const int slot = lane >> 1;
         if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
       }
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         float s, r;
         dev::block_scale(m, kEps, s, r);
         const uint64_t r2 = dev::splat2(r);
-        store_all(R, T, [&](int) { return r2; });
+        store_all(R, T, V, [&](int) { return r2; });
         if (lane == 0) *T.sdst = s;
     };
 

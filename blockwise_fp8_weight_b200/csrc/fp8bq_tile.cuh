@@ -122,24 +122,10 @@ struct TileCursor {
     }
 };
 
-// absmax bits of one 16-byte vector: a tree of three maxima (the integer
-// form needs sign-cleared first operands; the xorsign form ignores signs).
-template <int ESIZE>
-__device__ __forceinline__ uint32_t vec_absmax(const uint4 &v) {
-    constexpr uint32_t keep = FP8BQ_ABSMAX_FMAX ? 0xffffffffu : ESIZE == 2 ? 0x7fff7fffu
-                                                                          : 0x7fffffffu;
-    if constexpr (ESIZE == 2)
-        return dev::absmax_bf16x2(dev::absmax_bf16x2(v.x & keep, v.y),
-                                  dev::absmax_bf16x2(v.z & keep, v.w));
-    else
-        return dev::absmax_f32(dev::absmax_f32(v.x & keep, v.y), dev::absmax_f32(v.z & keep, v.w));
-}
-
 // absmax bits of V 16-byte vectors: four independent running maxima (one per
 // 32-bit lane of the vectors) so the max chains overlap, merged at the end.
 template <int ESIZE, int V>
 __device__ __forceinline__ uint32_t tile_absmax(const uint4 (&R)[V]) {
-    if constexpr (V == 1) return vec_absmax<ESIZE>(R[0]);
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
