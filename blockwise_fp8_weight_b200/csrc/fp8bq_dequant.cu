@@ -48,89 +48,96 @@ __device__ __forceinline__ const DequantDesc &find(const DequantPack<MAXD> &p, u
     return p.d[d];
 }
 
-// Vector kernel: a work item is a warp-wide row segment of 32 x U x 16 codes
-// (U 16-byte loads per lane, all issued before any is used; N and block_n are
-// multiples of 16, so the 16 codes of a load share one descale).  Items are
+// Vector kernel: a work item is a warp-wide row segment of 32 x U x 16 codes,
 // numbered row-major over (matrix, row, segment) and walked grid-stride by
-// warps, so index arithmetic is paid once per segment.
+// warps, so index arithmetic is paid once per segment.  A lane loads
+// 16 / OES codes at a time (8 for bf16 output, 4 for fp32), so each load
+// feeds exactly one 16-byte store and a warp store writes 512 contiguous
+// bytes, filling every sector it touches; all of a lane's loads of an item
+// are issued before any is used.  N and block_n are multiples of 16, so the
+// codes of one load share a descale.
 #ifndef FP8BQ_DQ_UNROLL
-#define FP8BQ_DQ_UNROLL 2  // measured: 1 -> 4.36, 2 -> 5.41, 4 -> 5.61 TB/s on one layer,
-                           // 4.64 / 5.58 / 5.48 TB/s on the whole weight set
+#define FP8BQ_DQ_UNROLL 4  // measured, fraction of the copy peak on one layer / the whole
+                           // weight set: 1 -> 0.62 / 0.62, 2 -> 0.82 / 0.86,
+                           // 4 -> 0.92-0.94 / 0.89-0.91, 8 -> 0.82 / 0.86
 #endif
-// Measured and dropped: 64 x 128 output tiles written into shared memory and
-// handed to TMA tile stores (72.9 M instructions on one layer, about the
-// same as here, and 121 us instead of 108 us cold; 0.69-0.72 of the copy
-// peak live against 0.84: two CTA barriers per tile and one issuing thread
-// serialise the tiles); numbering the items in 32 bits with shifts for
-// power-of-two blocks (43.9 M instead of 75.2 M instructions on one layer,
-// yet 142 us instead of 108 us: with the index arithmetic gone, nothing
-// hides the load latency -- long-scoreboard stalls 21 per issue against
-// 3.4), and one warp per whole row (4,199 / 3,889 GB/s against 5,499).
+// Measured and dropped: a lane loading 16 codes and writing them with two
+// 16-byte stores 32 bytes apart (each warp store half-fills 32 sectors; 0.84
+// of the copy peak on one layer and on the whole set); the same, software-
+// pipelined, with the next item's loads in flight while the current one is
+// decoded (0.71-0.75: more registers, fewer warps); 64 x 128 output tiles
+// written into shared memory and handed to TMA tile stores (0.69-0.72: two
+// CTA barriers per tile and one issuing thread serialise the tiles);
+// numbering the items in 32 bits with shifts for power-of-two blocks (with
+// the index arithmetic gone, nothing hides the load latency); one warp per
+// whole row (4,199 / 3,889 GB/s against 5,499 for the two-store form).
 constexpr int kDqUnroll = FP8BQ_DQ_UNROLL;
 
 template <int OES, int MAXD>
 __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ DequantPack<MAXD> p) {
     dev::pdl_entry();
-    constexpr int U = kDqUnroll;
+    constexpr int CPL = 16 / OES;              // codes per lane load
+    constexpr int L = kDqUnroll * 16 / CPL;    // loads per lane per item
     const int lane = threadIdx.x & 31;
     const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x >> 5);
     int d = 0;
     for (uint64_t k = (uint64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < p.total;
          k += warps) {
         const DequantDesc &a = find(p, k, d);
-        const int64_t n16 = a.N / 16;
-        const int64_t segs = (n16 + 32 * U - 1) / (32 * U);
+        const int64_t nc = a.N / CPL;
+        const int64_t segs = (nc + 32 * L - 1) / (32 * L);
         const int64_t local = (int64_t)(k - a.begin);
         const int64_t row_all = local / segs;            // b * M + r
-        const int64_t chunk0 = (local - row_all * segs) * 32 * U + lane;
-        if (chunk0 >= n16) continue;
+        const int64_t chunk0 = (local - row_all * segs) * 32 * L + lane;
+        if (chunk0 >= nc) continue;
         const int64_t b = row_all / a.M;
         const int64_t r = row_all - b * a.M;
         const uint8_t *src = a.y + row_all * a.N;
-        uint4 q[U];
+        uint32_t q[L][CPL / 4];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < L; ++u) {
             const int64_t chunk = chunk0 + 32 * u;
-            if (chunk < n16)
-                asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                             : "=r"(q[u].x), "=r"(q[u].y), "=r"(q[u].z), "=r"(q[u].w)
-                             : "l"(src + chunk * 16));
+            if (chunk < nc) {
+                if constexpr (CPL == 8)
+                    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
+                                 : "=r"(q[u][0]), "=r"(q[u][1])
+                                 : "l"(src + chunk * 8));
+                else
+                    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];"
+                                 : "=r"(q[u][0])
+                                 : "l"(src + chunk * 4));
+            }
         }
+        const float *srow = a.s + (b * a.gm + r / a.bm) * a.gn;
+        char *orow = (char *)a.out + ((b * a.obs) + r * a.ldo) * OES;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+        for (int u = 0; u < L; ++u) {
             const int64_t chunk = chunk0 + 32 * u;
-            if (chunk >= n16) break;
-            const int64_t c = chunk * 16;
-            const float s = __ldg(a.s + (b * a.gm + r / a.bm) * a.gn + c / a.bn);
+            if (chunk >= nc) break;
+            const int64_t c = chunk * CPL;
+            const float s = __ldg(srow + c / a.bn);
             uint64_t ss;
             asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
-            const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-            float v[16];
+            float v[CPL];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                decode2((uint16_t)(w[j] & 0xffffu), v[4 * j + 0], v[4 * j + 1]);
-                decode2((uint16_t)(w[j] >> 16), v[4 * j + 2], v[4 * j + 3]);
+            for (int j = 0; j < CPL / 4; ++j) {
+                decode2((uint16_t)(q[u][j] & 0xffffu), v[4 * j + 0], v[4 * j + 1]);
+                decode2((uint16_t)(q[u][j] >> 16), v[4 * j + 2], v[4 * j + 3]);
             }
 #pragma unroll
-            for (int j = 0; j < 8; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
-            char *dst = (char *)a.out + ((b * a.obs) + r * a.ldo + c) * OES;
+            for (int j = 0; j < CPL / 2; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
+            char *dst = orow + c * OES;
             if constexpr (OES == 2) {
-                uint32_t o[8];
+                uint32_t o[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+                for (int j = 0; j < 4; ++j) o[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
                 asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "r"(o[0]),
                              "r"(o[1]), "r"(o[2]), "r"(o[3])
                              : "memory");
-                asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16),
-                             "r"(o[4]), "r"(o[5]), "r"(o[6]), "r"(o[7])
-                             : "memory");
             } else {
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 16 * j),
-                                 "f"(v[4 * j]), "f"(v[4 * j + 1]), "f"(v[4 * j + 2]),
-                                 "f"(v[4 * j + 3])
-                                 : "memory");
+                asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v[0]),
+                             "f"(v[1]), "f"(v[2]), "f"(v[3])
+                             : "memory");
             }
         }
     }
