@@ -16,6 +16,11 @@ pages' Python API (verl docs "fp8_kernel.py -- FP8 量化内核", section 1 and
 
 They allocate the outputs with PyTorch (device memory and streams are
 PyTorch's job here) and hand the pointers to the library.
+
+With the environment variable ``FP8BQ_CHECKED=1`` set before the first call,
+the process loads ``libfp8bq_checked.so`` instead: the same library with every
+plain global access of its kernels bounds-checked (``fp8bq_checked_build``,
+``fp8bq_debug_take_bounds``).
 """
 from __future__ import annotations
 
@@ -25,7 +30,8 @@ import threading
 from typing import Iterable, Sequence
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libfp8bq.so")
+CHECKED = os.environ.get("FP8BQ_CHECKED", "0") not in ("", "0")
+LIB_PATH = os.path.join(_PKG, "libfp8bq_checked.so" if CHECKED else "libfp8bq.so")
 
 # fp8bq_dtype
 FP8BQ_BF16 = 0
@@ -42,12 +48,14 @@ FP8BQ_ERR_DEVICE_TIMEOUT = 7
 FP8BQ_ERR_ALIGN = 8
 FP8BQ_ERR_ARG = 9
 FP8BQ_ERR_DEVICE_UNSAFE = 10
+FP8BQ_ERR_DEVICE_BOUNDS = 11
 # fp8bq_path
 FP8BQ_PATH_AUTO = 0
 FP8BQ_PATH_VECTOR = 1
 FP8BQ_PATH_TMA = 2
 FP8BQ_PATH_GENERIC = 3
 FP8BQ_INJECT_DROP_FIRST_LOAD = 1
+FP8BQ_INJECT_TRIM_OUTPUTS = 2
 
 DEFAULT_BLOCK = (128, 128)
 
@@ -102,14 +110,15 @@ _lib = None
 
 
 def lib() -> ctypes.CDLL:
-    """Load ``libfp8bq.so`` (building it first with nvcc if it is missing or
-    older than its sources).  Raises if it cannot be built or loaded."""
+    """Load ``libfp8bq.so`` (``libfp8bq_checked.so`` under FP8BQ_CHECKED=1),
+    building it first with nvcc if it is missing or older than its sources.
+    Raises if it cannot be built or loaded."""
     global _lib
     with _lock:
         if _lib is None:
             from . import build as _build
-            if not _build.up_to_date():
-                _build.build()
+            if not _build.up_to_date(LIB_PATH):
+                _build.build(checked=CHECKED)
             L = ctypes.CDLL(LIB_PATH)
             vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             L.fp8bq_quantize.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, vp, vp]
@@ -144,6 +153,11 @@ def lib() -> ctypes.CDLL:
             L.fp8bq_debug_set_wait_limit_ns.restype = i32
             L.fp8bq_debug_set_inject.argtypes = [ctypes.c_uint32]
             L.fp8bq_debug_set_inject.restype = i32
+            L.fp8bq_checked_build.argtypes = []
+            L.fp8bq_checked_build.restype = i32
+            L.fp8bq_debug_take_bounds.argtypes = [ctypes.POINTER(ctypes.c_uint64),
+                                                  ctypes.POINTER(ctypes.c_uint64)]
+            L.fp8bq_debug_take_bounds.restype = i32
             _lib = L
     return _lib
 
@@ -259,6 +273,17 @@ def fp8bq_debug_set_wait_limit_ns(ns: int) -> int:
 
 def fp8bq_debug_set_inject(flags: int) -> int:
     return lib().fp8bq_debug_set_inject(flags)
+
+
+def fp8bq_checked_build() -> int:
+    return lib().fp8bq_checked_build()
+
+
+def fp8bq_debug_take_bounds() -> tuple[int, int, int]:
+    """``fp8bq_debug_take_bounds``: (status, count, first_address)."""
+    c, f = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    st = lib().fp8bq_debug_take_bounds(ctypes.byref(c), ctypes.byref(f))
+    return st, int(c.value), int(f.value)
 
 
 def check(status: int, what: str = "") -> None:

@@ -1,6 +1,9 @@
 """Build the in-tree shared library ``libfp8bq.so`` for sm_100a with nvcc.
 
-    python -m blockwise_fp8_weight_b200.build [--verbose-ptxas]
+    python -m blockwise_fp8_weight_b200.build [--verbose-ptxas] [--checked]
+
+``--checked`` builds ``libfp8bq_checked.so`` instead: the same library with
+every plain global access of its kernels bounds-checked (FP8BQ_CHECKED=1).
 
 The library links the CUDA runtime statically, so it does not depend on
 which libcudart the host process (e.g. PyTorch) loaded.
@@ -22,6 +25,7 @@ HEADERS = [os.path.join(CSRC, f) for f in ("fp8bq_internal.h", "fp8bq_device.cuh
                                                    "fp8bq_tile.cuh")] + [
     os.path.join(ROOT, "include", "fp8bq.h")]
 LIB = os.path.join(PKG, "libfp8bq.so")
+LIB_CHECKED = os.path.join(PKG, "libfp8bq_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-shared", "-Xcompiler", "-fPIC,-fvisibility=hidden",
@@ -37,20 +41,24 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
 
 
 def build(force: bool = False, verbose_ptxas: bool = False, out: str | None = None,
-          defines: tuple[str, ...] = ()) -> str:
+          defines: tuple[str, ...] = (), checked: bool = False) -> str:
     """Compile the library (to ``out``, default the in-tree path); ``defines``
-    are extra -D tuning constants."""
-    lib = out or LIB
-    if out is None and not force and not verbose_ptxas and not defines and up_to_date():
-        return LIB
+    are extra -D tuning constants; ``checked`` builds the bounds-checked
+    library (default path ``libfp8bq_checked.so``)."""
+    lib = out or (LIB_CHECKED if checked else LIB)
+    if checked:
+        defines = (*defines, "FP8BQ_CHECKED=1")
+    if out is None and not force and not verbose_ptxas and \
+            (checked or not defines) and up_to_date(lib):
+        return lib
     tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc(), *ARCH, *FLAGS, *(f"-D{d}" for d in defines), "-I", os.path.join(ROOT, "include"),
            "-o", tmp, *SOURCES]
@@ -65,6 +73,7 @@ if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--checked", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas, checked=a.checked))
     sys.exit(0)

@@ -343,6 +343,12 @@ uint64_t tiles_of(const fp8bq_desc &D, Variant v) {
            cdiv(cdiv(D.N, D.block_n), h);
 }
 
+// The extent the bounds checks of a checked build take for an output of
+// `bytes` bytes: one byte short under FP8BQ_INJECT_TRIM_OUTPUTS.
+[[maybe_unused]] uint64_t checked_out_extent(uint64_t bytes) {
+    return (g_inject.load() & FP8BQ_INJECT_TRIM_OUTPUTS) && bytes ? bytes - 1 : bytes;
+}
+
 void fill_tile_desc(const fp8bq_desc &D, Variant v, uint32_t begin, TileDesc *o) {
     o->x = D.x;
     o->y = D.y_u8;
@@ -359,6 +365,12 @@ void fill_tile_desc(const fp8bq_desc &D, Variant v, uint32_t begin, TileDesc *o)
     o->gn = (int32_t)cdiv(D.N, D.block_n);
     o->tile_begin = begin;
     o->tiles = (uint32_t)tiles_of(D, v);
+#if FP8BQ_CHECKED
+    const int64_t b1 = D.batch - 1;
+    o->x_bytes = (uint64_t)((b1 * o->xbs + (D.M - 1) * D.ld + D.N) * esize_of(D.dtype_in));
+    o->y_bytes = checked_out_extent((uint64_t)(b1 * o->ybs + D.M * D.N));
+    o->s_bytes = checked_out_extent((uint64_t)((b1 * o->sbs + (int64_t)o->gm * o->gn) * 4));
+#endif
 }
 
 template <int MAXD>
@@ -701,6 +713,12 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.items = vector ? (uint64_t)(D.batch * D.M) *
                                    (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
                              : (uint64_t)(D.batch * D.M * D.N);
+#if FP8BQ_CHECKED
+            o.y_bytes = (uint64_t)(D.batch * D.M * D.N);
+            o.s_bytes = (uint64_t)(D.batch * o.gm * (int64_t)o.gn * 4);
+            o.out_bytes = checked_out_extent(
+                (uint64_t)(((D.batch - 1) * o.obs + (D.M - 1) * D.ld_out + D.N) * oes));
+#endif
             p.total += o.items;
             ++p.n;
             ++i;
@@ -775,7 +793,7 @@ fp8bq_status run_dequant(const fp8bq_dequant_desc *t, int n, cudaStream_t stream
 
 template <int MAXD>
 cudaError_t launch_scale_group(const fp8bq_scale_desc *t, const std::vector<int> &idx, int es,
-                               float *scale_out, cudaStream_t st) {
+                               float *scale_out, uint64_t out_bytes, cudaStream_t st) {
     static thread_local ScalePack<MAXD> p;
     size_t i = 0;
     while (i < idx.size()) {
@@ -783,6 +801,7 @@ cudaError_t launch_scale_group(const fp8bq_scale_desc *t, const std::vector<int>
         p.pad_ = 0;
         p.total = 0;
         p.acc = reinterpret_cast<uint32_t *>(scale_out);
+        p.acc_bytes = out_bytes;
         while (i < idx.size() && p.n < MAXD) {
             const fp8bq_scale_desc &D = t[idx[i]];
             ScaleDesc &o = p.d[p.n];
@@ -823,7 +842,8 @@ fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out
     }
     const fp8bq_status sd = check_device();
     if (sd != FP8BQ_OK) return sd;
-    if (launch_scale_zero(scale_out, n, stream) != cudaSuccess) {
+    const uint64_t out_bytes = checked_out_extent((uint64_t)n * 4);
+    if (launch_scale_zero(scale_out, n, out_bytes, stream) != cudaSuccess) {
         cudaGetLastError();
         return FP8BQ_ERR_DEVICE;
     }
@@ -835,12 +855,30 @@ fp8bq_status run_tensor_scale(const fp8bq_scale_desc *t, int n, float *scale_out
         const int es = g ? 4 : 2;
         const cudaError_t e =
             groups[g].size() <= (size_t)kMaxDescSmall
-                ? launch_scale_group<kMaxDescSmall>(t, groups[g], es, scale_out, stream)
-                : launch_scale_group<kMaxDescLarge>(t, groups[g], es, scale_out, stream);
+                ? launch_scale_group<kMaxDescSmall>(t, groups[g], es, scale_out, out_bytes, stream)
+                : launch_scale_group<kMaxDescLarge>(t, groups[g], es, scale_out, out_bytes, stream);
         if (e != cudaSuccess) return FP8BQ_ERR_DEVICE;
     }
-    return launch_scale_finalize(scale_out, n, stream) == cudaSuccess ? FP8BQ_OK
-                                                                       : FP8BQ_ERR_DEVICE;
+    return launch_scale_finalize(scale_out, n, out_bytes, stream) == cudaSuccess
+               ? FP8BQ_OK
+               : FP8BQ_ERR_DEVICE;
+}
+
+// The bounds records of every kernel source file, summed (checked builds;
+// zeros without any CUDA call in a default build).
+cudaError_t bounds_records(uint64_t *count, uint64_t *first, bool clear) {
+    cudaError_t (*const fns[])(uint64_t *, uint64_t *, bool) = {
+        bounds_record_kernels, bounds_record_tma, bounds_record_dequant, bounds_record_scale};
+    *count = 0;
+    *first = 0;
+    for (auto fn : fns) {
+        uint64_t c = 0, f = 0;
+        const cudaError_t e = fn(&c, &f, clear);
+        if (e != cudaSuccess) return e;
+        *count += c;
+        if (*first == 0) *first = f;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -918,6 +956,9 @@ const char *fp8bq_status_string(fp8bq_status s) {
         case FP8BQ_ERR_DEVICE_UNSAFE:
             return "FP8BQ_ERR_DEVICE_UNSAFE: a kernel returned with a tile copy in flight; "
                    "stop using the GPU";
+        case FP8BQ_ERR_DEVICE_BOUNDS:
+            return "FP8BQ_ERR_DEVICE_BOUNDS: a checked kernel skipped an access outside its "
+                   "tensor";
     }
     return "FP8BQ_?: unknown status";
 }
@@ -933,7 +974,14 @@ fp8bq_status fp8bq_sync_status(cudaStream_t stream) {
         cudaGetLastError();
         return FP8BQ_ERR_DEVICE;
     }
-    return (w & 2u) ? FP8BQ_ERR_DEVICE_UNSAFE : w ? FP8BQ_ERR_DEVICE_TIMEOUT : FP8BQ_OK;
+    if (w & 2u) return FP8BQ_ERR_DEVICE_UNSAFE;
+    if (w) return FP8BQ_ERR_DEVICE_TIMEOUT;
+    uint64_t count = 0, first = 0;
+    if (bounds_records(&count, &first, false) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8BQ_ERR_DEVICE;
+    }
+    return count ? FP8BQ_ERR_DEVICE_BOUNDS : FP8BQ_OK;
 }
 
 int fp8bq_version(void) { return FP8BQ_VERSION; }
@@ -976,8 +1024,26 @@ fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns) {
 }
 
 fp8bq_status fp8bq_debug_set_inject(uint32_t flags) {
-    if (flags & ~FP8BQ_INJECT_DROP_FIRST_LOAD) return FP8BQ_ERR_ARG;
+    const uint32_t known =
+        FP8BQ_INJECT_DROP_FIRST_LOAD | (FP8BQ_CHECKED ? FP8BQ_INJECT_TRIM_OUTPUTS : 0u);
+    if (flags & ~known) return FP8BQ_ERR_ARG;
     g_inject.store(flags);
+    return FP8BQ_OK;
+}
+
+int fp8bq_checked_build(void) { return FP8BQ_CHECKED ? 1 : 0; }
+
+fp8bq_status fp8bq_debug_take_bounds(uint64_t *count, uint64_t *first_address) {
+    uint64_t c = 0, f = 0;
+    if (FP8BQ_CHECKED) {
+        if (check_device() != FP8BQ_OK) return FP8BQ_ERR_DEVICE;
+        if (cudaDeviceSynchronize() != cudaSuccess || bounds_records(&c, &f, true) != cudaSuccess) {
+            cudaGetLastError();
+            return FP8BQ_ERR_DEVICE;
+        }
+    }
+    if (count) *count = c;
+    if (first_address) *first_address = f;
     return FP8BQ_OK;
 }
 

@@ -40,6 +40,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return d;
 }
 
+// Byte ranges of a descriptor's codes, descales and output (the bounds checks
+// of checked builds; only ever expanded inside FP8BQ_IN).
+#define DQ_SPAN_Y(a) (dev::Span{(uint64_t)(a).y, (uint64_t)(a).y + (a).y_bytes})
+#define DQ_SPAN_S(a) (dev::Span{(uint64_t)(a).s, (uint64_t)(a).s + (a).s_bytes})
+#define DQ_SPAN_O(a) (dev::Span{(uint64_t)(a).out, (uint64_t)(a).out + (a).out_bytes})
+
 // Descriptor of work item k (items grow along each thread's grid-stride walk,
 // so the cursor only moves forward).
 template <int MAXD>
@@ -98,14 +104,18 @@ __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ Deq
         for (int u = 0; u < L; ++u) {
             const int64_t chunk = chunk0 + 32 * u;
             if (chunk < nc) {
-                if constexpr (CPL == 8)
+                if (!FP8BQ_IN(DQ_SPAN_Y(a), src + chunk * CPL, CPL)) {
+#pragma unroll
+                    for (int j = 0; j < CPL / 4; ++j) q[u][j] = 0;
+                } else if constexpr (CPL == 8) {
                     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];"
                                  : "=r"(q[u][0]), "=r"(q[u][1])
                                  : "l"(src + chunk * 8));
-                else
+                } else {
                     asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];"
                                  : "=r"(q[u][0])
                                  : "l"(src + chunk * 4));
+                }
             }
         }
         const float *srow = a.s + (b * a.gm + r / a.bm) * a.gn;
@@ -115,7 +125,8 @@ __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ Deq
             const int64_t chunk = chunk0 + 32 * u;
             if (chunk >= nc) break;
             const int64_t c = chunk * CPL;
-            const float s = __ldg(srow + c / a.bn);
+            const float *sp = srow + c / a.bn;
+            const float s = FP8BQ_IN(DQ_SPAN_S(a), sp, 4) ? __ldg(sp) : 0.0f;
             uint64_t ss;
             asm("mov.b64 %0, {%1, %1};" : "=l"(ss) : "f"(s));
             float v[CPL];
@@ -127,6 +138,7 @@ __global__ void __launch_bounds__(256) k_dequant_vec(const __grid_constant__ Deq
 #pragma unroll
             for (int j = 0; j < CPL / 2; ++j) mul2(v[2 * j], v[2 * j + 1], ss);
             char *dst = orow + c * OES;
+            if (!FP8BQ_IN(DQ_SPAN_O(a), dst, 16)) continue;
             if constexpr (OES == 2) {
                 uint32_t o[4];
 #pragma unroll
@@ -158,15 +170,18 @@ __global__ void __launch_bounds__(256)
         const int64_t rem = local - b * per_b;
         const int64_t r = rem / a.N;
         const int64_t c = rem - r * a.N;
-        const float s = __ldg(a.s + (b * a.gm + r / a.bm) * a.gn + c / a.bn);
+        const float *sp = a.s + (b * a.gm + r / a.bm) * a.gn + c / a.bn;
+        const float s = FP8BQ_IN(DQ_SPAN_S(a), sp, 4) ? __ldg(sp) : 0.0f;
         float v, unused;
-        decode2((uint16_t)__ldg(a.y + local), v, unused);
+        const uint8_t code = FP8BQ_IN(DQ_SPAN_Y(a), a.y + local, 1) ? __ldg(a.y + local) : 0;
+        decode2((uint16_t)code, v, unused);
         v = __fmul_rn(v, s);
-        const int64_t o = b * a.obs + r * a.ldo + c;
+        char *dst = (char *)a.out + (b * a.obs + r * a.ldo + c) * OES;
+        if (!FP8BQ_IN(DQ_SPAN_O(a), dst, OES)) continue;
         if constexpr (OES == 2)
-            ((uint16_t *)a.out)[o] = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xffffu);
+            *(uint16_t *)dst = (uint16_t)(pack_bf16x2(v, 0.0f) & 0xffffu);
         else
-            ((float *)a.out)[o] = v;
+            *(float *)dst = v;
     }
 }
 
@@ -194,5 +209,7 @@ template cudaError_t launch_dequant<kMaxDescSmall>(const DequantPack<kMaxDescSma
                                                    cudaStream_t);
 template cudaError_t launch_dequant<kMaxDescLarge>(const DequantPack<kMaxDescLarge> &, int, bool,
                                                    cudaStream_t);
+
+FP8BQ_DEFINE_BOUNDS_RECORD(bounds_record_dequant)
 
 }  // namespace fp8bq

@@ -33,6 +33,42 @@ __device__ __forceinline__ void prefetch_tensormap(const void *tmap) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
 
+// ---------------------------------------------------------------- checked builds
+//
+// With FP8BQ_CHECKED=1 every plain global load, store and atomic of the
+// kernels is first tested against the byte range of the tensor it belongs to
+// (FP8BQ_IN(span, address, bytes)); an access outside it is not made and is
+// recorded: a count and one address per translation unit and device.  The
+// default build compiles FP8BQ_IN to `true`, so its kernels are unchanged.
+#ifndef FP8BQ_CHECKED
+#define FP8BQ_CHECKED 0
+#endif
+
+// Byte range [lo, hi) of one tensor argument of a kernel.
+struct Span {
+    uint64_t lo, hi;
+};
+
+#if FP8BQ_CHECKED
+static __device__ unsigned long long g_bounds_count;
+static __device__ unsigned long long g_bounds_first;
+
+static __device__ __noinline__ void bounds_record(const void *p) {
+    atomicAdd(&g_bounds_count, 1ull);
+    atomicCAS(&g_bounds_first, 0ull, (unsigned long long)(uintptr_t)p);
+}
+
+__device__ __forceinline__ bool in_span(const Span &s, const void *p, uint64_t bytes) {
+    const uint64_t a = (uint64_t)(uintptr_t)p;
+    if (a >= s.lo && a <= s.hi && bytes <= s.hi - a) return true;
+    bounds_record(p);
+    return false;
+}
+#define FP8BQ_IN(span, p, bytes) (::fp8bq::dev::in_span((span), (p), (bytes)))
+#else
+#define FP8BQ_IN(span, p, bytes) true
+#endif
+
 // ---------------------------------------------------------------- global memory
 
 // 16-byte streaming load: read-only path, no L1 allocation, 256-byte L2
@@ -294,3 +330,33 @@ __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
 
 }  // namespace dev
 }  // namespace fp8bq
+
+// Host side of the bounds record: defines `cudaError_t fn(uint64_t *count,
+// uint64_t *first, bool clear)` reading (and, with clear, zeroing) this
+// translation unit's record on the current device; both are 0 in a default
+// build.  One use per kernel source file.
+#if FP8BQ_CHECKED
+#define FP8BQ_DEFINE_BOUNDS_RECORD(fn)                                                        \
+    cudaError_t fn(uint64_t *count, uint64_t *first, bool clear) {                             \
+        unsigned long long c = 0, f = 0;                                                       \
+        cudaError_t e = cudaMemcpyFromSymbol(&c, ::fp8bq::dev::g_bounds_count, sizeof(c));     \
+        if (e == cudaSuccess)                                                                  \
+            e = cudaMemcpyFromSymbol(&f, ::fp8bq::dev::g_bounds_first, sizeof(f));             \
+        if (e == cudaSuccess && clear && (c || f)) {                                           \
+            const unsigned long long zero = 0;                                                 \
+            e = cudaMemcpyToSymbol(::fp8bq::dev::g_bounds_count, &zero, sizeof(zero));         \
+            if (e == cudaSuccess)                                                              \
+                e = cudaMemcpyToSymbol(::fp8bq::dev::g_bounds_first, &zero, sizeof(zero));     \
+        }                                                                                      \
+        *count = c;                                                                            \
+        *first = f;                                                                            \
+        return e;                                                                              \
+    }
+#else
+#define FP8BQ_DEFINE_BOUNDS_RECORD(fn)                                                        \
+    cudaError_t fn(uint64_t *count, uint64_t *first, bool) {                                   \
+        *count = 0;                                                                            \
+        *first = 0;                                                                            \
+        return cudaSuccess;                                                                    \
+    }
+#endif

@@ -7,6 +7,10 @@
 
 #include <mutex>
 
+#ifndef FP8BQ_CHECKED
+#define FP8BQ_CHECKED 0  // 1: the bounds-checked build (see fp8bq_device.cuh)
+#endif
+
 namespace fp8bq {
 
 // ------------------------------------------------------------------ per-device host state
@@ -77,8 +81,11 @@ struct TileDesc {
     int32_t gm, gn;     // block grid of one matrix
     uint32_t tile_begin;// first tile id of this tensor within the launch
     uint32_t tiles;     // batch * gm * gn
+#if FP8BQ_CHECKED
+    uint64_t x_bytes, y_bytes, s_bytes;  // extents of x, y and s (the bounds checks)
+#endif
 };
-static_assert(sizeof(TileDesc) == 88, "TileDesc layout");
+static_assert(sizeof(TileDesc) == (FP8BQ_CHECKED ? 112 : 88), "TileDesc layout");
 
 // Grouped-launch parameters.  MAXD bounds the descriptors per launch so the
 // whole pack stays inside the 32 KB kernel-parameter limit.
@@ -109,7 +116,8 @@ struct alignas(64) TmaPack {
 constexpr uint64_t kEvictFirstMinBytes = 256ull << 20;
 
 constexpr int kMaxDescSmall = 8;
-constexpr int kMaxDescLarge = 320;  // 320 * 88 B + header = 28.2 KB
+// 320 * 88 B + header = 28.2 KB; checked builds 256 * 112 B + header = 28.7 KB
+constexpr int kMaxDescLarge = FP8BQ_CHECKED ? 256 : 320;
 constexpr int kMaxDescTma = 128;    // 128 * (128 + 88) B + header = 27.7 KB
 static_assert(sizeof(DescPack<kMaxDescLarge>) < 32000, "kernel parameter limit");
 static_assert(sizeof(TmaPack<kMaxDescTma>) < 32000, "kernel parameter limit");
@@ -172,8 +180,11 @@ struct DequantDesc {
     int32_t bm, bn, gm, gn;
     uint64_t begin;     // first work item of this descriptor
     uint64_t items;     // work items of this descriptor
+#if FP8BQ_CHECKED
+    uint64_t y_bytes, s_bytes, out_bytes;  // extents (the bounds checks)
+#endif
 };
-static_assert(sizeof(DequantDesc) == 88, "DequantDesc layout");
+static_assert(sizeof(DequantDesc) == (FP8BQ_CHECKED ? 112 : 88), "DequantDesc layout");
 
 template <int MAXD>
 struct DequantPack {
@@ -207,16 +218,25 @@ struct ScalePack {
     int32_t pad_;
     uint64_t total;
     uint32_t *acc;
+    uint64_t acc_bytes;  // extent of acc (the bounds checks of checked builds)
     ScaleDesc d[MAXD];
 };
 static_assert(sizeof(ScalePack<kMaxDescLarge>) < 32000, "kernel parameter limit");
 template <int MAXD>
 cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t st);
-cudaError_t launch_scale_zero(float *scale_out, int n, cudaStream_t st);
-cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st);
+// out_bytes: the extent of scale_out that the bounds checks of checked builds take
+cudaError_t launch_scale_zero(float *scale_out, int n, uint64_t out_bytes, cudaStream_t st);
+cudaError_t launch_scale_finalize(float *scale_out, int n, uint64_t out_bytes, cudaStream_t st);
 
 // Device error word access (fp8bq_tma.cu).
 cudaError_t read_and_clear_error_word(uint32_t *out);
+
+// Bounds records of checked builds, one per kernel source file (count of
+// skipped accesses, one of their addresses; both 0 in a default build).
+cudaError_t bounds_record_kernels(uint64_t *count, uint64_t *first, bool clear);
+cudaError_t bounds_record_tma(uint64_t *count, uint64_t *first, bool clear);
+cudaError_t bounds_record_dequant(uint64_t *count, uint64_t *first, bool clear);
+cudaError_t bounds_record_scale(uint64_t *count, uint64_t *first, bool clear);
 
 // Team geometry used by the vector kernels (host eligibility must agree).
 constexpr int kVecTeamThreads(Variant v, int esize) {

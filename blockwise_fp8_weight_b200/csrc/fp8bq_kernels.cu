@@ -137,11 +137,13 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
 
     // upper 8-byte half of this lane's vector inside the row (HALVES only)
     auto hi_ok = [&](const Tile &T) { return colv + VEC / 2 < T.cols; };
-    auto store = [&](const uint4 &v, uint64_t rr, uint8_t *dst, bool hi) {
-        if constexpr (HALVES)
-            vec_quant_store_halves<ESIZE>(v, rr, dst, hi);
-        else
-            vec_quant_store<ESIZE>(v, rr, dst);
+    auto store = [&](const Tile &T, const uint4 &v, uint64_t rr, uint8_t *dst, bool hi) {
+        if constexpr (HALVES) {
+            if (FP8BQ_IN(T.ys, dst, hi ? VEC : VEC / 2))
+                vec_quant_store_halves<ESIZE>(v, rr, dst, hi);
+        } else {
+            store_codes<ESIZE>(T, v, rr, dst);
+        }
     };
     // Every slot of every lane of the team lies inside the tile (the same for
     // the whole team): the interior tiles skip the per-vector bounds checks.
@@ -153,14 +155,14 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         const int64_t ystep = (int64_t)rstep * T.ldy;
         if (is_full(T)) {
 #pragma unroll
-            for (int i = 0; i < V; ++i) store(R[i], rr_of(i), dst + i * ystep, true);
+            for (int i = 0; i < V; ++i) store(T, R[i], rr_of(i), dst + i * ystep, true);
         } else {
             const bool hi = hi_ok(T);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 if (i >= nb) break;
                 if (row0 + i * rstep < T.rows && colv < T.cols)
-                    store(R[i], rr_of(i), dst + i * ystep, hi);
+                    store(T, R[i], rr_of(i), dst + i * ystep, hi);
             }
         }
     };
@@ -172,11 +174,12 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             if (r < T.rows && colv < T.cols) {
                 const char *a = T.src + ((int64_t)r * T.ld + colv) * ESIZE;
                 if constexpr (HALVES) {
-                    const uint2 lo = dev::ldg_v2(a);
-                    const uint2 hi = hi_ok(T) ? dev::ldg_v2(a + 8) : make_uint2(0u, 0u);
+                    const uint2 lo = FP8BQ_IN(T.xs, a, 8) ? dev::ldg_v2(a) : make_uint2(0u, 0u);
+                    const uint2 hi = hi_ok(T) && FP8BQ_IN(T.xs, a + 8, 8) ? dev::ldg_v2(a + 8)
+                                                                          : make_uint2(0u, 0u);
                     R[i] = make_uint4(lo.x, lo.y, hi.x, hi.y);
                 } else {
-                    R[i] = dev::ldg_stream_v4(a);
+                    R[i] = FP8BQ_IN(T.xs, a, 16) ? dev::ldg_stream_v4(a) : make_uint4(0u, 0u, 0u, 0u);
                 }
             } else {
                 R[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -211,7 +214,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         // slots of blocks below the matrix are neither quantized nor stored
         store_all(R, T, (T.rows + bm - 1) / bm, [&](int i) { return dev::splat2(r[i]); });
         const int slot = lane >> 1;
-        if ((lane & 1) == 0 && slot * bm < T.rows) T.sdst[(int64_t)slot * T.gn] = s_mine;
+        if ((lane & 1) == 0 && slot * bm < T.rows) store_descale(T, T.sdst + (int64_t)slot * T.gn, s_mine);
       }
     };
 
@@ -236,7 +239,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
         dev::block_scale(m, kEps, s, r);
         const uint64_t r2 = dev::splat2(r);
         store_all(R, T, V, [&](int) { return r2; });
-        if (lane == 0) *T.sdst = s;
+        if (lane == 0) store_descale(T, T.sdst, s);
     };
 
     if constexpr (S > 0) {
@@ -248,9 +251,10 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             const int64_t xstep = (int64_t)rstep * T.ld * ESIZE;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const bool ok = full || (row0 + i * rstep < T.rows && colv < T.cols);
-                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], ok ? src0 + i * xstep : T.src,
-                                 ok);
+                const char *src = src0 + i * xstep;
+                const bool ok = (full || (row0 + i * rstep < T.rows && colv < T.cols)) &&
+                                FP8BQ_IN(T.xs, src, 16);
+                dev::cp_async_16(&stage[(s * V + i) * CTA + threadIdx.x], ok ? src : T.src, ok);
             }
             dev::cp_async_commit();
         };
@@ -354,7 +358,9 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
         for (int r = 0; r < T.rows; ++r) {
             const char *row = T.src + (int64_t)r * T.ld * ESIZE;
 #pragma unroll 4
-            for (int c = lane; c < T.cols; c += 32) m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
+            for (int c = lane; c < T.cols; c += 32)
+                if (FP8BQ_IN(T.xs, row + c * ESIZE, ESIZE))
+                    m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
         }
         m = __reduce_max_sync(0xffffffffu, m);
         float s, rc;
@@ -364,11 +370,13 @@ __global__ void __launch_bounds__(256) k_generic(const __grid_constant__ DescPac
             uint8_t *out = T.dst + (int64_t)r * T.ldy;
 #pragma unroll 4
             for (int c = lane; c < T.cols; c += 32) {
-                const float v = __fmul_rn(elem_f32<ESIZE>(row + c * ESIZE), rc);
-                out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
+                const float x = FP8BQ_IN(T.xs, row + c * ESIZE, ESIZE) ? elem_f32<ESIZE>(row + c * ESIZE)
+                                                                      : 0.0f;
+                const float v = __fmul_rn(x, rc);
+                if (FP8BQ_IN(T.ys, out + c, 1)) out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
             }
         }
-        if (lane == 0) *T.sdst = s;
+        if (lane == 0) store_descale(T, T.sdst, s);
     }
 }
 
@@ -387,7 +395,9 @@ __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ Des
         for (int r = warp; r < T.rows; r += 8) {
             const char *row = T.src + (int64_t)r * T.ld * ESIZE;
 #pragma unroll 4
-            for (int c = lane; c < T.cols; c += 32) m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
+            for (int c = lane; c < T.cols; c += 32)
+                if (FP8BQ_IN(T.xs, row + c * ESIZE, ESIZE))
+                    m = max(m, elem_abs_bits<ESIZE>(row + c * ESIZE));
         }
         m = __reduce_max_sync(0xffffffffu, m);
         if (lane == 0) red[warp] = m;
@@ -403,11 +413,13 @@ __global__ void __launch_bounds__(256) k_generic_cta(const __grid_constant__ Des
             uint8_t *out = T.dst + (int64_t)r * T.ldy;
 #pragma unroll 4
             for (int c = lane; c < T.cols; c += 32) {
-                const float v = __fmul_rn(elem_f32<ESIZE>(row + c * ESIZE), rc);
-                out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
+                const float x = FP8BQ_IN(T.xs, row + c * ESIZE, ESIZE) ? elem_f32<ESIZE>(row + c * ESIZE)
+                                                                      : 0.0f;
+                const float v = __fmul_rn(x, rc);
+                if (FP8BQ_IN(T.ys, out + c, 1)) out[c] = (uint8_t)(dev::cvt_e4m3x2(v, 0.0f) & 0xffu);
             }
         }
-        if (threadIdx.x == 0) *T.sdst = s;
+        if (threadIdx.x == 0) store_descale(T, T.sdst, s);
     }
 }
 
@@ -484,5 +496,7 @@ template cudaError_t launch_generic<kMaxDescSmall>(int, const DescPack<kMaxDescS
                                                    cudaStream_t);
 template cudaError_t launch_generic<kMaxDescLarge>(int, const DescPack<kMaxDescLarge> &,
                                                    cudaStream_t);
+
+FP8BQ_DEFINE_BOUNDS_RECORD(bounds_record_kernels)
 
 }  // namespace fp8bq

@@ -20,7 +20,8 @@ namespace fp8bq {
 namespace {
 
 template <int ESIZE>
-__device__ __forceinline__ uint32_t elem_abs(const char *base, int64_t i) {
+__device__ __forceinline__ uint32_t elem_abs(const char *base, int64_t i, const dev::Span &xs) {
+    if (!FP8BQ_IN(xs, base + i * ESIZE, ESIZE)) return 0;
     if constexpr (ESIZE == 2)
         return ((uint32_t)__ldg((const unsigned short *)base + i) & 0x7fffu) << 16;
     else
@@ -30,14 +31,15 @@ __device__ __forceinline__ uint32_t elem_abs(const char *base, int64_t i) {
 // Fold a running max into the output slot of tensor `out`: CTA-wide reduce,
 // then one atomicMax (called when a CTA moves to another tensor and at the
 // end, so a tensor sees about one atomic per CTA).
-__device__ __forceinline__ void flush_max(uint32_t m, uint32_t *acc, int out, uint32_t *red) {
+__device__ __forceinline__ void flush_max(uint32_t m, uint32_t *acc, int out, uint32_t *red,
+                                          const dev::Span &accs) {
     m = __reduce_max_sync(0xffffffffu, m);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t t = red[0];
         for (int w = 1; w < 8; ++w) t = max(t, red[w]);
-        if (t) atomicMax(acc + out, t);
+        if (t && FP8BQ_IN(accs, acc + out, 4)) atomicMax(acc + out, t);
     }
     __syncthreads();
 }
@@ -50,10 +52,11 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
     __shared__ uint32_t red[8];
     int d = 0, cur = -1;
     uint32_t m = 0;
+    const dev::Span accs{(uint64_t)p.acc, (uint64_t)p.acc + p.acc_bytes};
     for (uint64_t it = blockIdx.x; it < p.total; it += gridDim.x) {
         while (it >= p.d[d].begin + p.d[d].items) ++d;
         if (d != cur) {  // uniform across the CTA: `it` is per CTA
-            if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red);
+            if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red, accs);
             m = 0;
             cur = d;
         }
@@ -61,11 +64,14 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
         const int64_t e0 = (int64_t)(it - D.begin) * kScaleItem;
         const int64_t len = min((int64_t)kScaleItem, D.numel - e0);
         const char *base = (const char *)D.x + e0 * ESIZE;
+        const dev::Span xs{(uint64_t)D.x, (uint64_t)D.x + (uint64_t)D.numel * ESIZE};
         if (len == kScaleItem && ((uintptr_t)base & 15) == 0) {
             uint4 v[LOADS];
 #pragma unroll
-            for (int j = 0; j < LOADS; ++j)
-                v[j] = dev::ldg_stream_v4(base + ((int64_t)j * 256 + threadIdx.x) * 16);
+            for (int j = 0; j < LOADS; ++j) {
+                const char *a = base + ((int64_t)j * 256 + threadIdx.x) * 16;
+                v[j] = FP8BQ_IN(xs, a, 16) ? dev::ldg_stream_v4(a) : make_uint4(0u, 0u, 0u, 0u);
+            }
 #pragma unroll
             for (int j = 0; j < LOADS; ++j) {
                 if constexpr (ESIZE == 2) {
@@ -79,23 +85,26 @@ __global__ void __launch_bounds__(256) k_scale_amax(const __grid_constant__ Scal
                 }
             }
         } else {
-            for (int64_t i = threadIdx.x; i < len; i += 256) m = max(m, elem_abs<ESIZE>(base, i));
+            for (int64_t i = threadIdx.x; i < len; i += 256) m = max(m, elem_abs<ESIZE>(base, i, xs));
         }
     }
-    if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red);
+    if (cur >= 0) flush_max(m, p.acc, p.d[cur].out, red, accs);
 }
 
 // Zero the accumulators (a kernel rather than a memset, so that the next
 // kernel of the chain can overlap its launch with this one).
-__global__ void k_scale_zero(float *scale_out, int n) {
+__global__ void k_scale_zero(float *scale_out, int n, uint64_t out_bytes) {
     dev::pdl_entry();
+    [[maybe_unused]] const dev::Span os{(uint64_t)scale_out, (uint64_t)scale_out + out_bytes};
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
-        scale_out[i] = 0.0f;
+        if (FP8BQ_IN(os, scale_out + i, 4)) scale_out[i] = 0.0f;
 }
 
-__global__ void k_scale_finalize(float *scale_out, int n) {
+__global__ void k_scale_finalize(float *scale_out, int n, uint64_t out_bytes) {
     dev::pdl_entry();
+    [[maybe_unused]] const dev::Span os{(uint64_t)scale_out, (uint64_t)scale_out + out_bytes};
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+        if (!FP8BQ_IN(os, scale_out + i, 4)) continue;
         const uint32_t bits = reinterpret_cast<const uint32_t *>(scale_out)[i];
         const float a = fmaxf(__uint_as_float(bits), kEps);
         scale_out[i] = __fdiv_rn(a, kFp8Max);
@@ -112,19 +121,23 @@ cudaError_t launch_scale_amax(const ScalePack<MAXD> &p, int esize, cudaStream_t 
                       : launch_kernel(k_scale_amax<4, MAXD>, grid, 256, 0, st, p);
 }
 
-cudaError_t launch_scale_zero(float *scale_out, int n, cudaStream_t st) {
+cudaError_t launch_scale_zero(float *scale_out, int n, uint64_t out_bytes, cudaStream_t st) {
     const int blocks = (n + 255) / 256;
-    return launch_kernel(k_scale_zero, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n);
+    return launch_kernel(k_scale_zero, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n,
+                         out_bytes);
 }
 
-cudaError_t launch_scale_finalize(float *scale_out, int n, cudaStream_t st) {
+cudaError_t launch_scale_finalize(float *scale_out, int n, uint64_t out_bytes, cudaStream_t st) {
     const int blocks = (n + 255) / 256;
-    return launch_kernel(k_scale_finalize, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n);
+    return launch_kernel(k_scale_finalize, blocks < 1 ? 1 : blocks, 256, 0, st, scale_out, n,
+                         out_bytes);
 }
 
 template cudaError_t launch_scale_amax<kMaxDescSmall>(const ScalePack<kMaxDescSmall> &, int,
                                                       cudaStream_t);
 template cudaError_t launch_scale_amax<kMaxDescLarge>(const ScalePack<kMaxDescLarge> &, int,
                                                       cudaStream_t);
+
+FP8BQ_DEFINE_BOUNDS_RECORD(bounds_record_scale)
 
 }  // namespace fp8bq

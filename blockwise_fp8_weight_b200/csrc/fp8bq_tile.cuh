@@ -19,6 +19,9 @@ struct Tile {
     int rows, cols;   // valid extent
     int b, bi, bj;    // coordinates (TMA)
     int gn;           // descale row length (blocks per matrix row)
+#if FP8BQ_CHECKED
+    dev::Span xs, ys, ss;  // byte ranges of the tensor's x, y and s
+#endif
 };
 
 // The tile whose first block is (bi, bj) of matrix b of descriptor D: grp
@@ -40,6 +43,11 @@ __device__ __forceinline__ Tile tile_at(const TileDesc &D, uint32_t b, uint32_t 
     T.bi = (int)bi;
     T.bj = (int)bj;
     T.gn = D.gn;
+#if FP8BQ_CHECKED
+    T.xs = {(uint64_t)D.x, (uint64_t)D.x + D.x_bytes};
+    T.ys = {(uint64_t)D.y, (uint64_t)D.y + D.y_bytes};
+    T.ss = {(uint64_t)D.s, (uint64_t)D.s + D.s_bytes};
+#endif
     return T;
 }
 
@@ -189,6 +197,18 @@ __device__ __forceinline__ void vec_quant_store(const uint4 &v, uint64_t rr, uin
     } else {
         dev::stg_stream_u32(dst, dev::quant_f32x4(v.x, v.y, v.z, v.w, rr));
     }
+}
+
+// The output stores of a tile (T: a Tile, or a kernel's own record of one
+// with the same fields): the codes of one 16-byte vector, and one descale.
+// In a checked build each is made only inside the tensor's byte range.
+template <int ESIZE, typename TT>
+__device__ __forceinline__ void store_codes(const TT &T, const uint4 &v, uint64_t rr, uint8_t *dst) {
+    if (FP8BQ_IN(T.ys, dst, 16 / ESIZE)) vec_quant_store<ESIZE>(v, rr, dst);
+}
+template <typename TT>
+__device__ __forceinline__ void store_descale(const TT &T, float *dst, float s) {
+    if (FP8BQ_IN(T.ss, dst, 4)) *dst = s;
 }
 
 // ------------------------------------------------------------------ grid sizing (host)

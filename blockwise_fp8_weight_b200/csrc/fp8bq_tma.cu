@@ -75,6 +75,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
         float *sdst;
         int64_t ldy;
         int32_t rows, cols, gn, pad;
+#if FP8BQ_CHECKED
+        dev::Span ys, ss;
+#endif
     };
     __shared__ SlotInfo info[STAGES];
     __shared__ __align__(8) uint64_t full[STAGES];
@@ -126,6 +129,10 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
             info[st].rows = T.rows;
             info[st].cols = T.cols;
             info[st].gn = p.d[d].gn;
+#if FP8BQ_CHECKED
+            info[st].ys = T.ys;
+            info[st].ss = T.ss;
+#endif
             dev::mbar_arrive_expect_tx(&full[st], tile_bytes);
             if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
                 dropped0 = true;  // fault injection: this slot's barrier can never complete
@@ -210,9 +217,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                 for (int i = 0; i < V; ++i) {
                     const int rr = row0 + i * rstep;
                     if (rr < T.rows && colv < T.cols)
-                        vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+                        store_codes<ESIZE>(T, R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
                 }
-                if (ct == 0) *T.sdst = s;
+                if (ct == 0) store_descale(T, T.sdst, s);
             } else {
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
@@ -225,9 +232,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                     dev::block_scale(m, kEps, s, r);
                     const int rr = row0 + i * rstep;
                     if (rr < T.rows && colv < T.cols)
-                        vec_quant_store<ESIZE>(R[i], dev::splat2(r),
-                                               T.dst + (int64_t)rr * T.ldy + colv);
-                    if (ct == 0 && i == j * spb) T.sdst[(int64_t)j * T.gn] = s;
+                        store_codes<ESIZE>(T, R[i], dev::splat2(r),
+                                           T.dst + (int64_t)rr * T.ldy + colv);
+                    if (ct == 0 && i == j * spb) store_descale(T, T.sdst + (int64_t)j * T.gn, s);
                 }
             }
         } else {
@@ -253,13 +260,13 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                 for (int i = 0; i < V; ++i) {
                     const int rr = row0 + i * rstep;
                     if (rr < T.rows && colv < T.cols)
-                        vec_quant_store<ESIZE>(R[i], dev::splat2(r[i]),
-                                               T.dst + (int64_t)rr * T.ldy + colv);
+                        store_codes<ESIZE>(T, R[i], dev::splat2(r[i]),
+                                           T.dst + (int64_t)rr * T.ldy + colv);
                 }
                 const int q = ct & (L - 1);  // this lane's block: slot q of its group
                 if (q < V) {
                     const int blk = (row0 + q * rstep) / bm;
-                    if (blk * bm < T.rows) T.sdst[(int64_t)blk * T.gn] = s_mine;
+                    if (blk * bm < T.rows) store_descale(T, T.sdst + (int64_t)blk * T.gn, s_mine);
                 }
             } else {
 #pragma unroll
@@ -270,9 +277,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
                     float s, r;
                     dev::block_scale(m[i], kEps, s, r);
                     if (rr < T.rows && colv < T.cols)
-                        vec_quant_store<ESIZE>(R[i], dev::splat2(r),
-                                               T.dst + (int64_t)rr * T.ldy + colv);
-                    if ((ct & (L - 1)) == 0) T.sdst[(int64_t)blk * T.gn] = s;
+                        store_codes<ESIZE>(T, R[i], dev::splat2(r),
+                                           T.dst + (int64_t)rr * T.ldy + colv);
+                    if ((ct & (L - 1)) == 0) store_descale(T, T.sdst + (int64_t)blk * T.gn, s);
                 }
             }
         }
@@ -307,6 +314,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
         float *sdst;
         int64_t ldy;
         int32_t rows, cols;
+#if FP8BQ_CHECKED
+        dev::Span ys, ss;
+#endif
     };
     __shared__ SlotInfo info[STAGES];
     __shared__ __align__(8) uint64_t full[STAGES];
@@ -354,6 +364,10 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
             info[st].ldy = T.ldy;
             info[st].rows = T.rows;
             info[st].cols = T.cols;
+#if FP8BQ_CHECKED
+            info[st].ys = T.ys;
+            info[st].ss = T.ss;
+#endif
             dev::mbar_arrive_expect_tx(&full[st], STAGE_BYTES);
             if ((p.inject & 1u) && blockIdx.x == 0 && k == 0)
                 dropped0 = true;
@@ -418,9 +432,9 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
         for (int i = 0; i < V; ++i) {
             const int rr = row0 + i * RSTEP;
             if (rr < T.rows && colv < T.cols)
-                vec_quant_store<ESIZE>(R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
+                store_codes<ESIZE>(T, R[i], r2, T.dst + (int64_t)rr * T.ldy + colv);
         }
-        if ((ct & 15) == 0 && ct < 32) T.sdst[half] = s;
+        if ((ct & 15) == 0 && ct < 32) store_descale(T, T.sdst + half, s);
     }
 }
 
@@ -495,5 +509,7 @@ cudaError_t read_and_clear_error_word(uint32_t *out) {
     if (*out) e = cudaMemcpyToSymbol(g_error_word, &zero, sizeof(uint32_t));
     return e;
 }
+
+FP8BQ_DEFINE_BOUNDS_RECORD(bounds_record_tma)
 
 }  // namespace fp8bq

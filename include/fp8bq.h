@@ -87,8 +87,10 @@ typedef enum fp8bq_status {
     FP8BQ_ERR_ALIGN = 8,          /* x not aligned to its element size, or descale not 4-byte
                                      aligned */
     FP8BQ_ERR_ARG = 9,            /* other invalid argument (n_tensors < 0, unknown path) */
-    FP8BQ_ERR_DEVICE_UNSAFE = 10  /* a kernel returned with a tile copy still in flight
+    FP8BQ_ERR_DEVICE_UNSAFE = 10, /* a kernel returned with a tile copy still in flight
                                      (reported by fp8bq_sync_status): stop using the GPU */
+    FP8BQ_ERR_DEVICE_BOUNDS = 11  /* checked builds only: a kernel skipped a global access
+                                     outside its tensor (reported by fp8bq_sync_status) */
 } fp8bq_status;
 
 /*
@@ -243,6 +245,11 @@ FP8BQ_API const char *fp8bq_status_string(fp8bq_status status);
  * a call reports (and clears) a timeout raised by a kernel on any stream of
  * the device, not only on `stream`, and whichever call reads it first takes
  * it.
+ *
+ * In a checked build (fp8bq_checked_build() == 1) it returns
+ * FP8BQ_ERR_DEVICE_BOUNDS, after the two statuses above, while the bounds
+ * record of the current device is not empty (see fp8bq_debug_take_bounds;
+ * this call does not clear it).
  */
 FP8BQ_API fp8bq_status fp8bq_sync_status(cudaStream_t stream);
 
@@ -311,10 +318,42 @@ FP8BQ_API int fp8bq_get_pdl(void);
  * the next TMA launches arm its first tile's barrier without issuing the
  * copy, so the consumers' wait can only run out; the kernel then reports
  * FP8BQ_ERR_DEVICE_TIMEOUT through fp8bq_sync_status.  0 turns it off.
+ *
+ * fp8bq_debug_set_inject(FP8BQ_INJECT_TRIM_OUTPUTS), in a checked build only
+ * (elsewhere FP8BQ_ERR_ARG), makes the bounds checks of the next launches
+ * take every output (codes, descales, dequantized values, per-tensor scales)
+ * as one byte shorter than its true extent, so the kernels' last, legitimate
+ * store to each output is reported and skipped: a test of the checks that
+ * touches no memory outside any buffer.  Flags combine with |.
  */
 #define FP8BQ_INJECT_DROP_FIRST_LOAD 1u
+#define FP8BQ_INJECT_TRIM_OUTPUTS 2u
 FP8BQ_API fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns);
 FP8BQ_API fp8bq_status fp8bq_debug_set_inject(uint32_t flags);
+
+/*
+ * Checked builds (library libfp8bq_checked.so, compiled with FP8BQ_CHECKED=1:
+ * a memory-safety aid for runs without a device sanitizer).  Every plain
+ * global load, store and atomic of every kernel is first tested against the
+ * byte range of the tensor it belongs to, taken from the call's descriptors:
+ * the input [x, x + ((batch - 1) x_batch_stride + (M - 1) ld + N) elements),
+ * the codes [y, y + (batch - 1) y_batch_stride + M N), the descales
+ * [s, s + ((batch - 1) s_batch_stride + gm gn) floats), and the like for the
+ * dequantizer and the per-tensor scales.  An access outside its range is not
+ * made (a load reads zeros) and is recorded per device: the number of such
+ * accesses and the address of one of them.  TMA tile loads are bounded by
+ * their tensor maps in hardware and are not checked.  Outputs are otherwise
+ * identical to the default build's; the checks cost speed, and the
+ * descriptor chunks per launch are smaller (256 instead of 320).
+ *
+ * fp8bq_checked_build returns 1 in a checked build, else 0.
+ * fp8bq_debug_take_bounds synchronizes the current device, stores the record
+ * (count of skipped accesses since the last take, and the address of one of
+ * them, 0 if none) and clears it; in a default build both are 0.  Either
+ * pointer may be NULL.  FP8BQ_ERR_DEVICE if the device cannot be read.
+ */
+FP8BQ_API int fp8bq_checked_build(void);
+FP8BQ_API fp8bq_status fp8bq_debug_take_bounds(uint64_t *count, uint64_t *first_address);
 
 #ifdef __cplusplus
 }

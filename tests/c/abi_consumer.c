@@ -26,7 +26,8 @@ int main(void) {
         (fn)fp8bq_sync_status,    (fn)fp8bq_version,          (fn)fp8bq_set_path,
         (fn)fp8bq_get_path,       (fn)fp8bq_path_for,         (fn)fp8bq_set_pdl,
         (fn)fp8bq_get_pdl,        (fn)fp8bq_debug_set_wait_limit_ns,
-        (fn)fp8bq_debug_set_inject, (fn)fp8bq_launch_count,
+        (fn)fp8bq_debug_set_inject, (fn)fp8bq_launch_count, (fn)fp8bq_checked_build,
+        (fn)fp8bq_debug_take_bounds,
     };
     size_t i;
     for (i = 0; i < sizeof entry / sizeof entry[0]; ++i) CHECK(entry[i] != NULL);
@@ -60,6 +61,14 @@ int main(void) {
     CHECK(fp8bq_get_pdl() == 1);
     CHECK(fp8bq_set_pdl(0) == FP8BQ_OK && fp8bq_get_pdl() == 0);
     CHECK(fp8bq_set_pdl(1) == FP8BQ_OK && fp8bq_get_pdl() == 1);
+    /* the default build: no bounds record, and the trimming knob is refused */
+    CHECK(fp8bq_checked_build() == 0);
+    CHECK(fp8bq_debug_set_inject(FP8BQ_INJECT_TRIM_OUTPUTS) == FP8BQ_ERR_ARG);
+    {
+        uint64_t count = 1, first = 1;
+        CHECK(fp8bq_debug_take_bounds(&count, &first) == FP8BQ_OK && count == 0 && first == 0);
+    }
+    CHECK(strlen(fp8bq_status_string(FP8BQ_ERR_DEVICE_BOUNDS)) > 0);
 
     printf("abi consumer ok\n");
     return 0;

@@ -48,7 +48,7 @@ def test_version_and_struct_layout():
 
 
 def test_status_strings():
-    for code in range(11):
+    for code in range(12):
         s = fq.fp8bq_status_string(code)
         assert s.startswith("FP8BQ_")
     assert "unknown" in fq.fp8bq_status_string(1234)
