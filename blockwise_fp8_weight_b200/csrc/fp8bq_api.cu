@@ -526,7 +526,41 @@ struct GroupKey {
 
 // The launches of one call: its tensors grouped by kernel variant (the
 // caller's order kept inside a group), with the TMA groups' tensor maps.
+// The same quantization on a geometry the kernels run better, for tensors of
+// at least kReshapeMinBytes of input with few rows (the result is identical
+// byte for byte; only the kernel's view changes):
+//  * a tensor of one block row (M <= block_m / 4) takes blocks of M rows: a
+//    block's absmax already covers only its M valid rows, and the descale
+//    grid (1 x gn) and code layout are unchanged;
+//  * row-wise blocks (block_m == 1) on fewer than kFoldRows contiguous rows
+//    (ld == N, N a multiple of block_n, one matrix) are refolded as k times
+//    more rows of N / k elements: every block keeps its elements, and both
+//    the codes and the descales keep their row-major order (block (r, j)
+//    becomes block (r k + j / (gn / k), j % (gn / k)), the same linear index).
+// Measured on B200 before this (bf16, one 2^27-element row): 1 x 128 blocks
+// 1.1 TB/s on the vector kernel (seven of the eight rows of its stacked tile
+// empty), 128 x 128 blocks 0.09 TB/s (one valid row in 128).
+constexpr uint64_t kReshapeMinBytes = 4ull << 20;
+constexpr int64_t kFoldRows = 256;
+
+fp8bq_desc reshaped(const fp8bq_desc &D) {
+    fp8bq_desc o = D;
+    if ((uint64_t)D.batch * (uint64_t)D.M * (uint64_t)D.N * esize_of(D.dtype_in) < kReshapeMinBytes)
+        return o;
+    if (o.M <= o.block_m / 4) o.block_m = (int32_t)o.M;
+    if (o.block_m == 1 && o.batch == 1 && o.ld == o.N && o.M < kFoldRows && o.N % o.block_n == 0) {
+        const int64_t gn = o.N / o.block_n;
+        int64_t k = 1;
+        while (o.M * k < kFoldRows && gn % (2 * k) == 0) k *= 2;
+        o.M *= k;
+        o.N /= k;
+        o.ld = o.N;
+    }
+    return o;
+}
+
 struct Plan {
+    std::vector<fp8bq_desc> descs;  // reshaped() of each tensor of the call
     std::vector<GroupKey> keys;
     std::vector<std::vector<int>> members;
     std::vector<std::vector<CUtensorMap>> maps;
@@ -551,6 +585,8 @@ fp8bq_status make_plan(const fp8bq_desc *table, int n, Plan &plan) {
     if (so != FP8BQ_OK) return so;
     const fp8bq_status sd = check_device();
     if (sd != FP8BQ_OK) return sd;
+    plan.descs.resize((size_t)n);
+    for (int i = 0; i < n; ++i) plan.descs[i] = empty[i] ? table[i] : reshaped(table[i]);
 
     // The kernel variant of each tensor.  AUTO sends a call's TMA tensors to
     // the vector kernel when together they hold less than kTmaMinCallBytes of
@@ -561,7 +597,7 @@ fp8bq_status make_plan(const fp8bq_desc *table, int n, Plan &plan) {
     uint64_t tma_bytes = 0;
     for (int i = 0; i < n; ++i) {
         if (empty[i]) continue;
-        const fp8bq_desc &D = table[i];
+        const fp8bq_desc &D = plan.descs[i];
         var[i] = choose(D, path);
         if (var[i] == Variant::Tma)
             tma_bytes += (uint64_t)D.batch * (uint64_t)D.M * (uint64_t)D.N * esize_of(D.dtype_in);
@@ -573,7 +609,7 @@ fp8bq_status make_plan(const fp8bq_desc *table, int n, Plan &plan) {
     std::vector<std::vector<CUtensorMap>> &maps = plan.maps;
     for (int i = 0; i < n; ++i) {
         if (empty[i]) continue;
-        const fp8bq_desc &D = table[i];
+        const fp8bq_desc &D = plan.descs[i];
         Variant v = var[i];
         CUtensorMap m;
         if (v == Variant::Tma && (small_call || !encode_map(D, &m)))
@@ -618,7 +654,8 @@ int packs_of(const fp8bq_desc *t, const std::vector<int> &idx, Variant v) {
     return packs;
 }
 
-int launches_of(const fp8bq_desc *table, const Plan &plan) {
+int launches_of(const Plan &plan) {
+    const fp8bq_desc *table = plan.descs.data();
     int total = 0;
     for (size_t g = 0; g < plan.keys.size(); ++g) {
         const std::vector<int> &idx = plan.members[g];
@@ -633,10 +670,11 @@ int launches_of(const fp8bq_desc *table, const Plan &plan) {
     return total;
 }
 
-fp8bq_status run(const fp8bq_desc *table, int n, cudaStream_t stream) {
+fp8bq_status run(const fp8bq_desc *caller_table, int n, cudaStream_t stream) {
     Plan plan;
-    const fp8bq_status sp = make_plan(table, n, plan);
+    const fp8bq_status sp = make_plan(caller_table, n, plan);
     if (sp != FP8BQ_OK || plan.keys.empty()) return sp;
+    const fp8bq_desc *table = plan.descs.data();
     const std::vector<GroupKey> &keys = plan.keys;
     const std::vector<std::vector<int>> &members = plan.members;
     const std::vector<std::vector<CUtensorMap>> &maps = plan.maps;
@@ -1005,7 +1043,7 @@ int fp8bq_path_for(const fp8bq_desc *desc) {
     if (desc == nullptr) return -1;
     bool e = false;
     if (check_desc(*desc, &e) != FP8BQ_OK) return -1;
-    switch (choose(*desc, g_path.load())) {
+    switch (choose(reshaped(*desc), g_path.load())) {
         case Variant::Tma: return FP8BQ_PATH_TMA;
         case Variant::Generic: return FP8BQ_PATH_GENERIC;
         default: return FP8BQ_PATH_VECTOR;
@@ -1015,7 +1053,7 @@ int fp8bq_path_for(const fp8bq_desc *desc) {
 int fp8bq_launch_count(const fp8bq_desc *desc_table, int n_tensors) {
     Plan plan;
     if (make_plan(desc_table, n_tensors, plan) != FP8BQ_OK) return -1;
-    return launches_of(desc_table, plan);
+    return launches_of(plan);
 }
 
 fp8bq_status fp8bq_debug_set_wait_limit_ns(uint64_t ns) {

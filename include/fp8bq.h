@@ -282,7 +282,11 @@ FP8BQ_API fp8bq_path fp8bq_get_path(void);
  * the descriptor is invalid.  This is the tensor's own choice; under AUTO a
  * call whose TMA tensors hold less than 128 MiB of input in all runs them on
  * the vector kernel (short launches start sooner there), which
- * fp8bq_launch_count accounts for.
+ * fp8bq_launch_count accounts for.  A tensor of at least 4 MiB of input with
+ * few rows is planned on an equivalent geometry with the same codes and
+ * descales (a single block row as blocks of its M rows; 1 x bn blocks on
+ * fewer than 256 contiguous rows folded into more, shorter rows), and the
+ * choice reported is the one for that geometry.
  */
 FP8BQ_API int fp8bq_path_for(const fp8bq_desc *desc);
 

@@ -94,7 +94,7 @@ typedef struct {
 typedef struct {
     const synth_spec *sp;
     void *out;
-    int64_t row_begin, row_end; /* over batch*M flattened rows */
+    int64_t el_begin, el_end; /* over the batch*M*N logical elements, row-major */
 } job;
 
 static double value_at(const synth_spec *sp, uint64_t kv, uint64_t kc, uint64_t ko,
@@ -130,7 +130,9 @@ static void *run_job(void *arg)
     uint64_t ko = stream_key(sp->seed, sp->tensor_id, TAG_OUTLIER);
     uint64_t kc = stream_key(sp->seed, sp->tensor_id, TAG_CHI);
     float pad = (float)sp->pad_value;
-    for (int64_t fr = jb->row_begin; fr < jb->row_end; ++fr) {
+    /* the rows this job's element range touches; a row's padding columns are
+     * written by the job that holds the row's last element */
+    for (int64_t fr = jb->el_begin / sp->N; fr * sp->N < jb->el_end; ++fr) {
         int64_t b = fr / sp->M, r = fr % sp->M;
         double factor = 1.0;
         if (sp->batch_lognormal_sigma != 0.0)
@@ -139,17 +141,20 @@ static void *run_job(void *arg)
             factor *= exp(sp->row_lognormal_sigma * normal_at(kr, (uint64_t)fr));
         int64_t base = b * sp->batch_stride + r * sp->ld;
         uint64_t e0 = (uint64_t)fr * (uint64_t)sp->N; /* logical element index */
+        int64_t c0 = jb->el_begin > fr * sp->N ? jb->el_begin - fr * sp->N : 0;
+        int64_t c1 = jb->el_end < (fr + 1) * sp->N ? jb->el_end - fr * sp->N : sp->N;
+        int64_t p1 = c1 == sp->N ? sp->ld : c1;
         if (sp->dtype == 0) {
             uint16_t *o = (uint16_t *)jb->out + base;
-            for (int64_t c = 0; c < sp->N; ++c)
+            for (int64_t c = c0; c < c1; ++c)
                 o[c] = bf16_rne((float)value_at(sp, kv, kc, ko, factor, e0 + (uint64_t)c));
-            for (int64_t c = sp->N; c < sp->ld; ++c)
+            for (int64_t c = c1; c < p1; ++c)
                 o[c] = bf16_rne(pad);
         } else {
             float *o = (float *)jb->out + base;
-            for (int64_t c = 0; c < sp->N; ++c)
+            for (int64_t c = c0; c < c1; ++c)
                 o[c] = (float)value_at(sp, kv, kc, ko, factor, e0 + (uint64_t)c);
-            for (int64_t c = sp->N; c < sp->ld; ++c)
+            for (int64_t c = c1; c < p1; ++c)
                 o[c] = pad;
         }
     }
@@ -165,18 +170,34 @@ int synth_fill(const synth_spec *sp, void *out)
     int64_t rows = sp->batch * sp->M;
     if (rows == 0 || sp->ld == 0)
         return 0;
+    if (sp->N == 0) { /* rows of padding only */
+        for (int64_t fr = 0; fr < rows; ++fr) {
+            int64_t base = (fr / sp->M) * sp->batch_stride + (fr % sp->M) * sp->ld;
+            for (int64_t c = 0; c < sp->ld; ++c) {
+                if (sp->dtype == 0)
+                    ((uint16_t *)out)[base + c] = bf16_rne((float)sp->pad_value);
+                else
+                    ((float *)out)[base + c] = (float)sp->pad_value;
+            }
+        }
+        return 0;
+    }
+    /* threads split the logical elements evenly (values depend only on the
+     * element's index, so any split gives the same array): long rows of
+     * few-row tensors are shared too */
+    int64_t total = rows * sp->N;
     int nt = sp->nthreads < 1 ? 1 : sp->nthreads;
     if (nt > 256)
         nt = 256;
-    if (nt > rows)
-        nt = (int)rows;
+    if (total < (int64_t)nt * 4096)
+        nt = (int)(total / 4096) > 0 ? (int)(total / 4096) : 1;
     pthread_t th[256];
     job jobs[256];
     for (int t = 0; t < nt; ++t) {
         jobs[t].sp = sp;
         jobs[t].out = out;
-        jobs[t].row_begin = rows * t / nt;
-        jobs[t].row_end = rows * (t + 1) / nt;
+        jobs[t].el_begin = (int64_t)((__int128)total * t / nt);
+        jobs[t].el_end = (int64_t)((__int128)total * (t + 1) / nt);
     }
     int started = 0;
     for (int t = 1; t < nt; ++t) {

@@ -116,3 +116,33 @@ def assert_same(spec: TensorSpec, got, want) -> None:
     sb = np.flatnonzero(sg.view(np.uint32).reshape(-1) != sw.view(np.uint32).reshape(-1))
     assert sb.size == 0, (f"{spec.name}: {sb.size} descales differ; first at {sb[0]}: got "
                           f"{sg.reshape(-1)[sb[0]]!r} want {sw.reshape(-1)[sb[0]]!r}")
+
+
+def sample_blocks(sp: TensorSpec, rng, k=6):
+    gm, gn = sp.grid
+    picks = {(0, 0, 0), (sp.batch - 1, gm - 1, gn - 1), (0, 0, gn - 1), (sp.batch - 1, gm - 1, 0)}
+    for _ in range(k):
+        picks.add((int(rng.integers(sp.batch)), int(rng.integers(gm)), int(rng.integers(gn))))
+    return sorted(picks)
+
+
+def check_sampled(sp: TensorSpec, x: np.ndarray, out: Outputs, rng, k=6) -> int:
+    """Compare sampled blocks of a device output with the oracle, block by block."""
+    gm, gn = sp.grid
+    bm, bn = sp.block
+    yv = out.y.view.view(sp.batch, sp.M, sp.N)
+    sv = out.s.view.view(torch.float32).view(sp.batch, gm, gn)
+    n = 0
+    for b, bi, bj in sample_blocks(sp, rng, k):
+        xb = np.ascontiguousarray(x[b * sp.batch_stride:(b + 1) * sp.batch_stride])
+        yw, sw = oracle.quantize_block(xb, sp.M, sp.N, sp.row_stride, bm, bn, bi, bj)
+        yg = yv[b, bi * bm:bi * bm + yw.shape[0], bj * bn:bj * bn + yw.shape[1]].cpu().numpy()
+        sg = float(sv[b, bi, bj].item())
+        assert np.array_equal(yg, yw), (sp.name, b, bi, bj, int((yg != yw).sum()))
+        assert np.float32(sg).view(np.uint32) == np.float32(sw).view(np.uint32), (sp.name, b, bi, bj)
+        n += 1
+    return n
+
+
+def no_nan_codes(out: Outputs) -> bool:
+    return not bool(((out.y.view & 0x7F) == 0x7F).any().item())

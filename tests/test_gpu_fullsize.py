@@ -25,7 +25,7 @@ import oracle
 from synth import TensorSpec
 from synth import workloads as W
 from tests import oracle_pool as OP
-from tests.gpu_util import Outputs, run, to_device
+from tests.gpu_util import check_sampled, no_nan_codes, run, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -56,36 +56,6 @@ def offsets(sizes) -> tuple[list[int], int]:
         out.append(o)
         o = align(o + n)
     return out, o
-
-
-def sample_blocks(sp: TensorSpec, rng, k=6):
-    gm, gn = sp.grid
-    picks = {(0, 0, 0), (sp.batch - 1, gm - 1, gn - 1), (0, 0, gn - 1), (sp.batch - 1, gm - 1, 0)}
-    for _ in range(k):
-        picks.add((int(rng.integers(sp.batch)), int(rng.integers(gm)), int(rng.integers(gn))))
-    return sorted(picks)
-
-
-def check_sampled(sp: TensorSpec, x: np.ndarray, out: Outputs, rng, k=6) -> int:
-    """Compare sampled blocks of a device output with the oracle, block by block."""
-    gm, gn = sp.grid
-    bm, bn = sp.block
-    yv = out.y.view.view(sp.batch, sp.M, sp.N)
-    sv = out.s.view.view(torch.float32).view(sp.batch, gm, gn)
-    n = 0
-    for b, bi, bj in sample_blocks(sp, rng, k):
-        xb = np.ascontiguousarray(x[b * sp.batch_stride:(b + 1) * sp.batch_stride])
-        yw, sw = oracle.quantize_block(xb, sp.M, sp.N, sp.row_stride, bm, bn, bi, bj)
-        yg = yv[b, bi * bm:bi * bm + yw.shape[0], bj * bn:bj * bn + yw.shape[1]].cpu().numpy()
-        sg = float(sv[b, bi, bj].item())
-        assert np.array_equal(yg, yw), (sp.name, b, bi, bj, int((yg != yw).sum()))
-        assert np.float32(sg).view(np.uint32) == np.float32(sw).view(np.uint32), (sp.name, b, bi, bj)
-        n += 1
-    return n
-
-
-def no_nan_codes(out: Outputs) -> bool:
-    return not bool(((out.y.view & 0x7F) == 0x7F).any().item())
 
 
 class HostSet:

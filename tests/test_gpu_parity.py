@@ -160,6 +160,32 @@ def test_degenerate_shapes_and_blocks(shape, block, dtype):
     del owner
 
 
+@pytest.mark.parametrize("shape,block,dtype,ld", [
+    ((1, 1 << 22), (1, 128), "bf16", None),        # 8 MB: folded into 256 rows
+    ((1, 1 << 22), (128, 128), "bf16", None),      # one block row: blocks of 1 row, folded
+    ((3, 3 << 20), (1, 128), "f32", None),         # folded by 2^k while gn allows
+    ((8, 1 << 20), (128, 128), "bf16", None),      # blocks of 8 rows
+    ((2, (1 << 21) + 64), (1, 64), "bf16", None),  # gn odd: no fold
+    ((4, 1 << 20), (64, 128), "bf16", 1 << 20 | 64),  # padded rows: blocks of 4 rows, no fold
+    ((40, 1 << 18), (128, 128), "bf16", None),     # more than a quarter block: unchanged
+])
+def test_few_row_tensors(shape, block, dtype, ld):
+    """Tensors of a few rows, which the planner runs on an equivalent geometry
+    (blocks of their M rows, row-wise blocks folded into more rows): every
+    code and descale against the oracle, on every path."""
+    M, N = shape
+    sp = TensorSpec(f"few.{M}x{N}.b{block}", M, N, block=block, dtype=dtype, ld=ld, seed=73,
+                    tensor_id=M * 131 + block[0], dist=DIST_STUDENT_T3, row_lognormal_sigma=1.0)
+    x = W.materialize(sp)
+    owner, ptr = to_device(x)
+    want = oracle_expected(sp, x)
+    for path in PATHS.values():
+        (o,) = run([sp], [ptr], path)
+        assert_same(sp, o.result(), want)
+        assert fq.fp8bq_launch_count([o.desc(ptr)]) == 1
+    del owner
+
+
 def test_all_zero_and_one_element_blocks():
     sp = TensorSpec("zeros", 200, 264, seed=0)
     x = np.zeros(sp.numel_storage, dtype=np.uint16)
