@@ -32,10 +32,16 @@
  * the current device).  The library writes only y and descale, allocates no
  * device memory per call, and keeps no pointer after a call returns.
  *
- * Devices: a process drives one GPU (one process per GPU, as under torchrun).
- * The library raises its kernels' dynamic shared-memory limit, and sizes
- * their grids, on the first device that launches them; calls made later on
- * another device of the same process are not supported.
+ * Devices: a call runs on the current CUDA device, whose memory its pointers
+ * must name.  Everything the library sets up for a device (the kernels'
+ * dynamic shared-memory limits, resident CTAs per SM, the SM count, its own
+ * streams for concurrent launch groups) is made once per device with that
+ * device current, so one process may use several GPUs, in turn or at once.
+ *
+ * Threads: every entry point may be called from several host threads at
+ * once, on the same or different streams and devices.  The process-wide
+ * settings (fp8bq_set_path, fp8bq_set_pdl and the debug knobs) are shared by
+ * all threads; change them while no call is being made.
  *
  * Execution: calls are asynchronous on `stream`, like a kernel launch.  All
  * arguments are checked before anything is launched: a call that returns an

@@ -377,6 +377,43 @@ def test_concurrent_groups_keep_stream_order(edge_case):
                              sc.cpu().numpy().view(np.float32).reshape(sp.batch, gm, gn)), w)
 
 
+def test_calls_from_several_host_threads(edge_case, qwen_layer_case):
+    """Four host threads call the library at once, each on its own stream
+    (the ctypes calls release the GIL, so the library's planning, tensor-map
+    cache and launch-group fork run concurrently): every output of every
+    thread is the oracle's."""
+    import threading
+    from tests.gpu_util import Outputs
+    cases = [edge_case, qwen_layer_case, edge_case, qwen_layer_case]
+    outs = [[Outputs(sp) for sp in c.specs] for c in cases]
+    descs = [[o.desc(p) for o, p in zip(oo, c.ptrs)] for oo, c in zip(outs, cases)]
+    streams = [torch.cuda.Stream() for _ in cases]
+    errors = []
+    start = threading.Barrier(len(cases))
+
+    def work(k):
+        try:
+            start.wait()
+            for _ in range(10):
+                st = fq.fp8bq_quantize_batched(descs[k], stream=streams[k])
+                assert st == fq.FP8BQ_OK, fq.fp8bq_status_string(st)
+            assert fq.fp8bq_sync_status(streams[k]) == fq.FP8BQ_OK
+        except BaseException as e:                       # reported below
+            errors.append((k, repr(e)))
+
+    threads = [threading.Thread(target=work, args=(k,)) for k in range(len(cases))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=300)
+    assert not any(t.is_alive() for t in threads)
+    assert not errors, errors
+    torch.cuda.synchronize()
+    for c, oo in zip(cases, outs):
+        for sp, o, w in zip(c.specs, oo, c.want):
+            assert_same(sp, o.result(), w)
+
+
 def test_mixed_variant_call_in_a_cuda_graph(edge_case):
     """Under graph capture the launch groups of a call stay on the capturing
     stream; replays write the oracle's bytes."""
