@@ -747,7 +747,7 @@ cudaError_t launch_dequant_group(const fp8bq_dequant_desc *t, const std::vector<
             o.gm = (int32_t)cdiv(D.M, D.block_m);
             o.gn = (int32_t)cdiv(D.N, D.block_n);
             o.begin = p.total;
-            // vector: warp items of 32 x 16 codes per row; generic: one element
+            // vector: warp items of 32 x U x 16 codes per row; generic: one element
             o.items = vector ? (uint64_t)(D.batch * D.M) *
                                    (uint64_t)cdiv(D.N / 16, 32 * dequant_unroll())
                              : (uint64_t)(D.batch * D.M * D.N);

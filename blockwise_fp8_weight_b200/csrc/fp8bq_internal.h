@@ -170,8 +170,8 @@ cudaError_t launch_tma_pair(const TmaPack<MAXD> &p, cudaStream_t st);
 
 // Dequantization (fp8bq_dequant.cu): one matrix stack per descriptor, a
 // grouped launch walks the concatenated work items (a warp-wide row segment
-// of 32 x 16 codes for the vector kernel, one element for the generic one) of
-// all descriptors of a pack.
+// of 32 x U x 16 codes for the vector kernel, U = dequant_unroll(); one
+// element for the generic one) of all descriptors of a pack.
 struct DequantDesc {
     const uint8_t *y;   // [batch, M, N] codes
     const float *s;     // [batch, gm, gn] descales
@@ -197,7 +197,7 @@ static_assert(sizeof(DequantPack<kMaxDescLarge>) < 32000, "kernel parameter limi
 
 template <int MAXD>
 cudaError_t launch_dequant(const DequantPack<MAXD> &p, int out_esize, bool vector, cudaStream_t st);
-// 16-byte code chunks per lane in a work item of the vector dequant kernel
+// U: a work item of the vector dequant kernel holds U x 16 codes per lane
 int dequant_unroll();
 
 // Per-tensor scales (fp8bq_scale.cu): the tensors of a pack are cut into
