@@ -205,11 +205,35 @@ __device__ __forceinline__ uint32_t absmax_bits_f32(uint32_t m) { return m & 0x7
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Scale and reciprocal of a block from the bit pattern of its fp32 absmax.
+// Scale and reciprocal of a block from the bit pattern of its fp32 absmax:
+// s = a / 448 and r = 1 / s, both correctly rounded (IEEE round to nearest).
+//
+// FP8BQ_DIV448_FMA 1: the division by the constant 448 as a multiply by
+// z = RN(1/448) and one FMA correction, q0 = RN(a z), s = RN(q0 + RN(a - 448 q0) z)
+// (the remainder a - 448 q0 is exact under the FMA): the division by a divisor
+// known in advance of Brisebarre, Muller and Raina ("Accelerating correctly
+// rounded floating-point division when the divisor is known in advance",
+// IEEE Trans. Computers 53(8), 2004), which is correctly rounded for every
+// dividend only for some divisors.  For 448 it has been checked against IEEE
+// division for every float a >= 1e-10 (the eps floor; tests/c/div448_check.c,
+// 1.35e9 values, no difference).  The reciprocal is __frcp_rn, itself
+// correctly rounded.  Measured on B200 against two IEEE divisions: 1.6 % fewer
+// instructions for 1 x 128 blocks, +0.3-1.5 % on the small-block and ragged
+// lines, one layer 0.997 against 0.991-0.995 of the copy peak.
+#ifndef FP8BQ_DIV448_FMA
+#define FP8BQ_DIV448_FMA 1
+#endif
 __device__ __forceinline__ void block_scale(uint32_t amax_bits, float eps, float &s, float &r) {
     float a = fmaxf(__uint_as_float(amax_bits), eps);
+#if FP8BQ_DIV448_FMA
+    constexpr float z = 1.0f / 448.0f;
+    const float q0 = __fmul_rn(a, z);
+    s = __fmaf_rn(__fmaf_rn(-q0, 448.0f, a), z, q0);
+    r = __frcp_rn(s);
+#else
     s = __fdiv_rn(a, 448.0f);
     r = __fdiv_rn(1.0f, s);
+#endif
 }
 
 // ---------------------------------------------------------------- timers, barriers
