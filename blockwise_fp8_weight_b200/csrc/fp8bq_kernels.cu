@@ -26,6 +26,22 @@
 namespace fp8bq {
 
 // Tuning constants (compile-time; the defaults are the measured best on B200).
+// Grid cap of the vector kernel in waves of resident CTAs: the team-of-16
+// kernel (stacked small blocks) runs two, the others one.  Measured on B200
+// (same box, one wave / two / three, fraction of the copy peak): [1,128]
+// blocks 0.86-0.88 / 0.93-0.94 / 0.90; [64,64] blocks 0.95 / 0.95 / 0.93;
+// bf16 4096x4096 0.94 / 0.96-0.97 / 0.84; bf16 4000x4100 0.80 / 0.83 / 0.75,
+// sixteen of them in one call 0.86 / 0.81 / 0.83; the per-tensor loop over
+// the Qwen3-8B-shaped weight set 0.830 / 0.816 / 0.79 -- a second wave of
+// short-lived CTAs evens out the SMs' finishing times of some launches and
+// costs others their ring's warm-up, so only the 1 x 128 case, which gains
+// most, takes it.
+#ifndef FP8BQ_VEC_WAVES
+#define FP8BQ_VEC_WAVES 1
+#endif
+#ifndef FP8BQ_VEC_WAVES_T16
+#define FP8BQ_VEC_WAVES_T16 2
+#endif
 #ifndef FP8BQ_VEC_CTAS_PER_SM
 #define FP8BQ_VEC_CTAS_PER_SM 2   // resident 256-thread vector CTAs per SM
 #endif
@@ -435,7 +451,8 @@ cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
     static PerDevice<KernelSetup> setup;
     const KernelSetup ks = setup.get([&] { return setup_kernel(kern, CTA, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, ks.occ);
+    constexpr int waves = TEAM == 16 ? FP8BQ_VEC_WAVES_T16 : FP8BQ_VEC_WAVES;
+    const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, ks.occ * waves);
     return launch_kernel(kern, grid, CTA, smem, st, p);
 }
 

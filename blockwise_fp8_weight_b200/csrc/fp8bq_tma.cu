@@ -6,6 +6,10 @@
 // on an mbarrier is bounded; a wait that runs out sets the device error word.
 #include "fp8bq_tile.cuh"
 
+#ifndef FP8BQ_TMA_WAVES
+#define FP8BQ_TMA_WAVES 1  // grid cap in waves of resident CTAs
+#endif
+
 namespace fp8bq {
 
 // Bit 0: a consumer or producer wait ran out (that launch's outputs are
@@ -449,7 +453,7 @@ cudaError_t launch_tma_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     const KernelSetup ks =
         setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ), 32 + kTmaConsumerThreads,
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES), 32 + kTmaConsumerThreads,
                          smem, st, p);
 }
 
@@ -470,7 +474,7 @@ cudaError_t launch_tma_pair_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     const KernelSetup ks =
         setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ), 32 + kTmaConsumerThreads,
+    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES), 32 + kTmaConsumerThreads,
                          smem, st, p);
 }
 }  // namespace
