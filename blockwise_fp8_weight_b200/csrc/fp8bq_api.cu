@@ -550,8 +550,12 @@ fp8bq_desc reshaped(const fp8bq_desc &D) {
     if (o.M <= o.block_m / 4) o.block_m = (int32_t)o.M;
     if (o.block_m == 1 && o.batch == 1 && o.ld == o.N && o.M < kFoldRows && o.N % o.block_n == 0) {
         const int64_t gn = o.N / o.block_n;
+        const int64_t es = esize_of(o.dtype_in);
         int64_t k = 1;
-        while (o.M * k < kFoldRows && gn % (2 * k) == 0) k *= 2;
+        // folded rows stay a whole number of 16-byte vectors if the rows were
+        while (o.M * k < kFoldRows && gn % (2 * k) == 0 &&
+               ((o.N * es) % 16 != 0 || (o.N / (2 * k) * es) % 16 == 0))
+            k *= 2;
         o.M *= k;
         o.N /= k;
         o.ld = o.N;
