@@ -168,7 +168,7 @@ def test_degenerate_shapes_and_blocks(shape, block, dtype):
     ((2, (1 << 21) + 64), (1, 64), "bf16", None),  # gn odd: no fold
     ((4, 1 << 20), (64, 128), "bf16", 1 << 20 | 64),  # padded rows: blocks of 4 rows, no fold
     ((40, 1 << 18), (128, 128), "bf16", None),     # more than a quarter block: unchanged
-    ((1, 3 << 20), (1, 4), "bf16", None),          # folded only while rows stay 16-byte vectors
+    ((1, 64 * 32769), (1, 4), "bf16", None),       # folded by 8, not 16: rows stay 16-byte vectors
 ])
 def test_few_row_tensors(shape, block, dtype, ld):
     """Tensors of a few rows, which the planner runs on an equivalent geometry
