@@ -6,8 +6,21 @@
 // on an mbarrier is bounded; a wait that runs out sets the device error word.
 #include "fp8bq_tile.cuh"
 
+// Grid cap of the TMA kernels in waves of resident CTAs.  Measured on B200
+// (same box), two / four waves against one: the whole weight set +0.5 / +1.2 %,
+// one layer -0.5 / -3.5 %, the MoE layer -1.5 / -1.2 %: one wave, a
+// persistent walk.
 #ifndef FP8BQ_TMA_WAVES
-#define FP8BQ_TMA_WAVES 1  // grid cap in waves of resident CTAs
+#define FP8BQ_TMA_WAVES 1
+#endif
+// Resident CTAs per SM of the paired kernel (its register budget follows).
+// Measured on B200 (same box): two CTAs of one 64 KB slot each (96
+// registers) against one CTA of two slots: one layer 0.935-0.939 / 0.984-0.994,
+// the whole weight set 0.959 / 0.988-0.989, the MoE layer 0.966-0.974 /
+// 1.002-1.006 of the copy peak -- a CTA that overlaps its own next load with
+// its current tile beats two that each wait for theirs.
+#ifndef FP8BQ_TMA_PAIR_CTAS_PER_SM
+#define FP8BQ_TMA_PAIR_CTAS_PER_SM 1
 #endif
 
 namespace fp8bq {
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_CTAS_PER_S
 #endif
 
 template <int STAGES, int MAXD, bool EF>
-__global__ void __launch_bounds__(32 + kTmaConsumerThreads, 1)
+__global__ void __launch_bounds__(32 + kTmaConsumerThreads, FP8BQ_TMA_PAIR_CTAS_PER_SM)
     k_tma_pair(const __grid_constant__ TmaPack<MAXD> P) {
     dev::pdl_launch_dependents();
     constexpr int ESIZE = 2, VEC = 8, BN = 128, BM = 128;
@@ -453,8 +466,8 @@ cudaError_t launch_tma_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     const KernelSetup ks =
         setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES), 32 + kTmaConsumerThreads,
-                         smem, st, p);
+    const unsigned grid = grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES);
+    return launch_kernel(kern, grid, 32 + kTmaConsumerThreads, smem, st, p);
 }
 
 // The L2 policy of the tile loads is a template parameter, so the default
@@ -474,8 +487,8 @@ cudaError_t launch_tma_pair_e(const TmaPack<MAXD> &p, cudaStream_t st) {
     const KernelSetup ks =
         setup.get([&] { return setup_kernel(kern, 32 + kTmaConsumerThreads, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    return launch_kernel(kern, grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES), 32 + kTmaConsumerThreads,
-                         smem, st, p);
+    const unsigned grid = grid_for(p.p.total_tiles, 1, ks.occ * FP8BQ_TMA_WAVES);
+    return launch_kernel(kern, grid, 32 + kTmaConsumerThreads, smem, st, p);
 }
 }  // namespace
 
