@@ -38,8 +38,12 @@ constexpr uint64_t kDrainLimitNs = 2000000000ull;
 #ifndef FP8BQ_TMA_STAGES_BF16
 #define FP8BQ_TMA_STAGES_BF16 4   // 32 KB ring slots per TMA CTA (bf16 tiles)
 #endif
+// 64 KB ring slots per TMA CTA (fp32 tiles).  Measured on B200 (one fp32
+// Qwen3-8B-shaped layer / four in one call, fraction of the copy peak):
+// 3 slots 0.937-0.944 / 0.954-0.957, 2 slots 1.028-1.030 / 1.048-1.049; as
+// for the paired bf16 kernel, a third 64 KB slot per SM slows the stream.
 #ifndef FP8BQ_TMA_STAGES_F32
-#define FP8BQ_TMA_STAGES_F32 3    // 64 KB ring slots per TMA CTA (fp32 tiles)
+#define FP8BQ_TMA_STAGES_F32 2
 #endif
 #ifndef FP8BQ_TMA_CTAS_PER_SM
 #define FP8BQ_TMA_CTAS_PER_SM 1   // resident TMA CTAs per SM
