@@ -77,9 +77,10 @@ __device__ __forceinline__ int first_desc(const DequantPack<MAXD> &p, uint64_t k
 // are issued before any is used.  N and block_n are multiples of 16, so the
 // codes of one load share a descale.
 #ifndef FP8BQ_DQ_UNROLL
-#define FP8BQ_DQ_UNROLL 4  // measured with a grid of 8 CTAs per SM, fraction of the copy
-                           // peak on one layer / the whole weight set: 1 -> 0.62 / 0.62,
-                           // 2 -> 0.82 / 0.86, 4 -> 0.92-0.94 / 0.89-0.91, 8 -> 0.82 / 0.86
+#define FP8BQ_DQ_UNROLL 4  // measured, fraction of the copy peak on one layer / the whole
+                           // weight set: grid of 8 CTAs per SM: 1 -> 0.62 / 0.62, 2 -> 0.82 /
+                           // 0.86, 4 -> 0.92-0.94 / 0.89-0.91, 8 -> 0.82 / 0.86; grid of 32
+                           // per SM: 2 -> 0.86 / 0.83, 4 -> 0.96 / 0.97, 8 -> 0.81 / 0.82
 #endif
 // Measured and dropped: a lane loading 16 codes and writing them with two
 // 16-byte stores 32 bytes apart (each warp store half-fills 32 sectors; 0.84
