@@ -376,8 +376,14 @@ def scaled_fp8_blockwise(data_hp, weight_block_size=DEFAULT_BLOCK, stream=None):
     _check_cuda(data_hp, "data_hp")
     with _on_stream(stream):
         y, s = _outputs(data_hp, block)
-    check(fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream),
-          "scaled_fp8_blockwise")
+    if data_hp.dim() == 2 and (data_hp.shape[-1] <= 1 or data_hp.stride(-1) == 1):
+        M, N = data_hp.shape
+        ld = max(data_hp.stride(0) if M > 1 else max(N, 1), N)
+        st = lib().fp8bq_quantize(data_hp.data_ptr(), _dtype_code(data_hp), M, N, ld, block[0],
+                                  block[1], y.data_ptr(), s.data_ptr(), _stream(stream))
+    else:
+        st = fp8bq_quantize_batched([make_desc(data_hp, y, s, block)], stream=stream)
+    check(st, "scaled_fp8_blockwise")
     return y, s
 
 
@@ -427,21 +433,75 @@ def tensor_scales(tensors, stream=None):
     return out
 
 
+# fp8bq_desc as a numpy record (the same 96-byte layout), so that a whole
+# table is built from one list of tuples instead of field by field.
+_DESC_RECORD = [("x", "<u8"), ("y_u8", "<u8"), ("descale_f32", "<u8"), ("M", "<i8"),
+                ("N", "<i8"), ("ld", "<i8"), ("batch", "<i8"), ("x_batch_stride", "<i8"),
+                ("y_batch_stride", "<i8"), ("s_batch_stride", "<i8"), ("dtype_in", "<i4"),
+                ("block_m", "<i4"), ("block_n", "<i4"), ("reserved", "<i4")]
+
+
+def _plan_weights(named, bm: int, bn: int, stream=None):
+    """Descriptor table (a numpy record array) and output views of
+    quant_weights: the fp8 weights are views of one allocation and the
+    descales of another, each piece at a 256-byte aligned offset."""
+    import numpy as np
+    import torch
+    cur = torch.cuda.current_device() if torch.cuda.is_available() else -1
+    rows = []
+    yo = so = 0
+    for name, w in named:
+        if not isinstance(w, torch.Tensor) or not w.is_cuda or w.device.index != cur:
+            _check_cuda(w, name)  # raises with the reason
+        shape = w.shape
+        if len(shape) not in (2, 3):
+            raise ValueError(f"{name}: expected a 2-D weight or a 3-D stack of expert weights")
+        M, N = shape[-2], shape[-1]
+        if N > 1 and w.stride(-1) != 1:
+            raise ValueError(f"{name}: the last dimension of the input must have unit stride")
+        dt = FP8BQ_BF16 if w.dtype == torch.bfloat16 else _dtype_code(w)
+        gm, gn = -(-M // bm), -(-N // bn)
+        stack = len(shape) == 3
+        E = shape[0] if stack else 1
+        rows.append((w, shape, yo, so, gm, gn, E, M, N, stack, dt))
+        yo += (E * M * N + 255) & ~255
+        so += (E * gm * gn + 63) & ~63
+    dev = named[0][1].device
+    with _on_stream(stream):
+        ybuf = torch.empty(max(yo, 1), dtype=torch.uint8, device=dev).view(torch.float8_e4m3fn)
+        sbuf = torch.empty(max(so, 1), dtype=torch.float32, device=dev)
+    yp, sp = ybuf.data_ptr(), sbuf.data_ptr()
+    recs, outs = [], []
+    for (name, _w), (w, shape, yoff, soff, gm, gn, E, M, N, stack, dt) in zip(named, rows):
+        ld = max(w.stride(-2) if M > 1 else max(N, 1), N)
+        recs.append((w.data_ptr(), yp + yoff, sp + 4 * soff, M, N, ld, E,
+                     w.stride(0) if stack else 0, M * N if stack else 0,
+                     gm * gn if stack else 0, dt, bm, bn, 0))
+        if stack:
+            y = ybuf.as_strided((E, M, N), (M * N, N, 1), yoff)
+            s = sbuf.as_strided((E, gm, gn), (gm * gn, gn, 1), soff)
+        else:
+            y = ybuf.as_strided((M, N), (N, 1), yoff)
+            s = sbuf.as_strided((gm, gn), (gn, 1), soff)
+        outs.append((name, y))
+        outs.append((name + "_scale_inv", s))
+    return np.array(recs, dtype=_DESC_RECORD), outs
+
+
 def quant_weights(weights: Iterable, weight_block_size=DEFAULT_BLOCK, stream=None):
     """Quantize every (name, tensor) pair in one grouped call and return the
     list the rollout engine loads: (name, fp8 weight) followed by
-    (name + "_scale_inv", descale) for each input, in input order."""
-    block = tuple(int(b) for b in weight_block_size)
-    items, descs = [], []
-    for name, w in weights:
-        _check_cuda(w, name)
-        with _on_stream(stream):
-            y, s = _outputs(w, block)
-        items.append((name, y, s, w))
-        descs.append(make_desc(w, y, s, block))
-    check(fp8bq_quantize_batched(descs, stream=stream), "quant_weights")
-    out = []
-    for name, y, s, _w in items:
-        out.append((name, y))
-        out.append((name + "_scale_inv", s))
+    (name + "_scale_inv", descale) for each input, in input order.
+
+    The fp8 weights are views of one device allocation and the descales of
+    another (each piece at a 256-byte aligned offset), so a whole model costs
+    two allocations; the memory is returned when the last view is freed."""
+    bm, bn = (int(b) for b in weight_block_size)
+    named = list(weights)
+    if not named:
+        return []
+    table, out = _plan_weights(named, bm, bn, stream)
+    st = lib().fp8bq_quantize_batched(table.ctypes.data_as(ctypes.POINTER(fp8bq_desc)),
+                                      len(named), _stream(stream))
+    check(st, "quant_weights")
     return out

@@ -47,6 +47,17 @@ def test_version_and_struct_layout():
     assert fq.fp8bq_desc.block_n.offset == 88
 
 
+def test_numpy_descriptor_record_matches_the_struct():
+    """quant_weights builds its descriptor table as a numpy record array: the
+    same size and field offsets as struct fp8bq_desc."""
+    import numpy as np
+    rec = np.dtype(fq._DESC_RECORD)
+    assert rec.itemsize == ctypes.sizeof(fq.fp8bq_desc)
+    assert [n for n, _ in fq._DESC_RECORD] == [n for n, _ in fq.fp8bq_desc._fields_]
+    for name, _ in fq._DESC_RECORD:
+        assert rec.fields[name][1] == getattr(fq.fp8bq_desc, name).offset, name
+
+
 def test_status_strings():
     for code in range(12):
         s = fq.fp8bq_status_string(code)

@@ -230,6 +230,43 @@ def test_non_default_stream_and_python_api():
     assert torch.equal(out[3][1], d[:4])
 
 
+def test_quant_weights_mixed_list_against_the_oracle():
+    """quant_weights over a mixed list (bf16 and fp32, an expert stack, a
+    ragged shape, a column slice with row padding): one grouped call whose
+    outputs are views of two shared allocations; every byte and descale
+    against the oracle, every view disjoint from the others."""
+    specs = [
+        TensorSpec("w.a", 1024, 4096, seed=77, tensor_id=1, row_lognormal_sigma=0.5),
+        TensorSpec("w.b", 130, 129, seed=77, tensor_id=2, dist=DIST_STUDENT_T3),
+        TensorSpec("w.c", 256, 384, dtype="f32", seed=77, tensor_id=3),
+        TensorSpec("w.d", 512, 768, batch=4, seed=77, tensor_id=4, batch_lognormal_sigma=0.7),
+        TensorSpec("w.e", 300, 200, ld=264, seed=77, tensor_id=5),
+    ]
+    tens, wants = [], []
+    for sp in specs:
+        x = W.materialize(sp)
+        wants.append(oracle_expected(sp, x))
+        dt = torch.bfloat16 if sp.dtype == "bf16" else torch.float32
+        raw = torch.from_numpy(x.view(np.int16) if sp.dtype == "bf16" else x).view(dt).cuda()
+        t = raw.reshape(sp.batch, sp.M, sp.row_stride)[..., :sp.N]
+        tens.append(t if sp.batch > 1 else t[0])
+    out = fq.quant_weights([(sp.name, t) for sp, t in zip(specs, tens)])
+    torch.cuda.synchronize()
+    assert [n for n, _ in out] == [n for sp in specs for n in (sp.name, sp.name + "_scale_inv")]
+    spans = []
+    for i, sp in enumerate(specs):
+        y, d = out[2 * i][1], out[2 * i + 1][1]
+        assert y.dtype == torch.float8_e4m3fn and y.shape == tens[i].shape and y.is_contiguous()
+        gm, gn = sp.grid
+        assert d.shape == ((sp.batch, gm, gn) if sp.batch > 1 else (gm, gn))
+        assert_same(sp, (y.view(torch.uint8).cpu().numpy().reshape(sp.batch, sp.M, sp.N),
+                         d.cpu().numpy().reshape(sp.batch, gm, gn)), wants[i])
+        for t in (y, d):
+            spans.append((t.data_ptr(), t.data_ptr() + t.numel() * t.element_size()))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+
+
 def test_expert_stack_python_api():
     sp = W.moe_layer(3)[5]                             # w2 [128, 2048, 768]
     sp = TensorSpec(sp.name, sp.M, sp.N, batch=8, seed=sp.seed, tensor_id=sp.tensor_id,
