@@ -42,6 +42,17 @@ namespace fp8bq {
 #ifndef FP8BQ_VEC_WAVES_T16
 #define FP8BQ_VEC_WAVES_T16 2
 #endif
+// Short launches of the other vector kernels (fewer than 8 tiles per
+// resident team) take two waves as well: measured on B200 (same box, one
+// wave / two), bf16 4096x4096 0.93 / 0.95-0.97, the edge set 0.88 / 0.89-0.90,
+// bf16 4000x4100 0.79-0.80 / 0.77-0.82; the long launches keep one wave
+// (sixteen 4000x4100, [64,64] blocks and the per-tensor loop unchanged).
+#ifndef FP8BQ_VEC_WAVES_SHORT
+#define FP8BQ_VEC_WAVES_SHORT 2
+#endif
+#ifndef FP8BQ_VEC_SHORT_TILES
+#define FP8BQ_VEC_SHORT_TILES 8
+#endif
 #ifndef FP8BQ_VEC_CTAS_PER_SM
 #define FP8BQ_VEC_CTAS_PER_SM 2   // resident 256-thread vector CTAs per SM
 #endif
@@ -455,7 +466,13 @@ cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
     static PerDevice<KernelSetup> setup;
     const KernelSetup ks = setup.get([&] { return setup_kernel(kern, CTA, smem); });
     if (ks.attr != cudaSuccess) return ks.attr;
-    constexpr int waves = TEAM == 16 ? FP8BQ_VEC_WAVES_T16 : FP8BQ_VEC_WAVES;
+    // short launches (fewer than FP8BQ_VEC_SHORT_TILES tiles per resident
+    // team) take FP8BQ_VEC_WAVES_SHORT waves
+    const uint64_t resident_teams = (uint64_t)sm_count() * ks.occ * (CTA / TEAM);
+    const int waves = TEAM == 16 ? FP8BQ_VEC_WAVES_T16
+                      : p.total_tiles < (uint64_t)FP8BQ_VEC_SHORT_TILES * resident_teams
+                          ? FP8BQ_VEC_WAVES_SHORT
+                          : FP8BQ_VEC_WAVES;
     const unsigned grid = grid_for(p.total_tiles, CTA / TEAM, ks.occ * waves);
     return launch_kernel(kern, grid, CTA, smem, st, p);
 }
