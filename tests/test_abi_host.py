@@ -47,6 +47,23 @@ def test_version_and_struct_layout():
     assert fq.fp8bq_desc.block_n.offset == 88
 
 
+@pytest.mark.parametrize("M,N,block,path", [
+    (1, 1 << 22, (128, 128), fq.FP8BQ_PATH_VECTOR),  # 8 MB, one row: 1-row blocks, folded
+    (1, 1024, (128, 128), fq.FP8BQ_PATH_TMA),        # 2 KB: below the size, planned as given
+    (8, 1 << 20, (128, 128), fq.FP8BQ_PATH_VECTOR),  # blocks of its 8 rows
+    (40, 1 << 18, (128, 128), fq.FP8BQ_PATH_TMA),    # more than a quarter block: as given
+    (1, 1 << 22, (1, 128), fq.FP8BQ_PATH_VECTOR),
+])
+def test_few_row_planning_without_a_device(M, N, block, path):
+    """fp8bq_path_for reports the variant of the planner's equivalent geometry
+    for few-row tensors of at least 4 MiB (host only, no device needed)."""
+    d = fq.fp8bq_desc()
+    d.x, d.y_u8, d.descale_f32 = X, Y, S
+    d.M, d.N, d.ld, d.batch = M, N, N, 1
+    d.dtype_in, (d.block_m, d.block_n) = fq.FP8BQ_BF16, block
+    assert fq.fp8bq_path_for(d) == path
+
+
 def test_numpy_descriptor_record_matches_the_struct():
     """quant_weights builds its descriptor table as a numpy record array: the
     same size and field offsets as struct fp8bq_desc."""
