@@ -600,7 +600,10 @@ def run_ours(args) -> None:
     l2_mb = torch.cuda.get_device_properties(dev).L2_cache_size / 1e6
     launch_s = elapsed_s / args.steps / max(launches, 1)
     achieved = bytes_per_step / max(launches, 1) / launch_s / 1e9
-    traffic, traffic_source = traffic_for(args.workload, args.path, launches)
+    # the records are of the grouped call (one call per step); other modes run
+    # other launches, so they report no traffic
+    traffic, traffic_source = traffic_for(args.workload, args.path, launches) \
+        if args.mode == "grouped" and args.repeat == 1 else (None, None)
 
     if rank == 0:
         line = {
