@@ -654,15 +654,16 @@ def run_ours(args) -> None:
 
 
 def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_desc) -> None:
-    """Time fp8bq_dequantize_batched (bf16 output) over every quantized tensor
-    of the workload, one grouped call per step; the codes come from the
-    quantize steps already run."""
+    """Time fp8bq_dequantize_batched (bf16 output, or fp32 with --dq-out f32)
+    over every quantized tensor of the workload, one grouped call per step;
+    the codes come from the quantize steps already run."""
     import torch
     import blockwise_fp8_weight_b200 as fq
+    oes = 4 if args.dq_out == "f32" else 2
     out_off, o = [], 0
     for sp in specs:
         out_off.append(o)
-        o = align(o + sp.numel * 2, 256)
+        o = align(o + sp.numel * oes, 256)
     out = torch.empty(o, dtype=torch.uint8, device=dev)
     L = fq.lib()
     stream = torch.cuda.current_stream(dev)
@@ -675,7 +676,7 @@ def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_de
         d.out = out.data_ptr() + out_off[i]
         d.batch, d.M, d.N = sp.batch, sp.M, sp.N
         d.ld_out, d.out_batch_stride = sp.N, sp.M * sp.N
-        d.dtype_out = fq.FP8BQ_BF16
+        d.dtype_out = fq.FP8BQ_F32 if oes == 4 else fq.FP8BQ_BF16
         d.block_m, d.block_n = sp.block
         d.reserved = 0
 
@@ -700,18 +701,18 @@ def run_dequant_op(args, specs, lay, y_dev, s_dev, dev, dist, world, rank, wl_de
         torch.cuda.synchronize()
     dist.barrier()
     el = dist.max(t0.elapsed_time(t1) / 1e3)
-    nbytes = sum(sp.numel * 3 + sp.nblocks * 4 for sp in specs)
+    nbytes = sum(sp.numel * (1 + oes) + sp.nblocks * 4 for sp in specs)
     value = aggregate(nbytes, args.steps, world, el)
     peak, kind = measured_peak()
     dq_launches = -(-len(specs) // 320)  # 320 descriptors per launch
     if rank == 0:
         print(json.dumps({
-            "metric": "blockwise FP8 dequantize GB/s (e4m3 codes + descales in, bf16 out)",
+            "metric": f"blockwise FP8 dequantize GB/s (e4m3 codes + descales in, {args.dq_out} out)",
             "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": wl_desc + " (dequantize its codes to bf16)",
+            "config": {"workload": wl_desc + f" (dequantize its codes to {args.dq_out})",
                        "name": args.workload, "op": "dequantize", "bytes_per_step": nbytes,
                        "launches_per_step": dq_launches, "path": args.path},
             "roofline": {"bound": "hbm", "achieved": value / world, "peak": peak, "unit": "GB/s",
@@ -910,6 +911,8 @@ def main() -> None:
     ap.add_argument("--mode", choices=["grouped", "per_layer", "per_tensor"], default="grouped",
                     help="C-ABI calls per step: one grouped call, one per layer, or one per "
                          "tensor")
+    ap.add_argument("--dq-out", choices=["bf16", "f32"], default="bf16",
+                    help="output dtype of --op dequantize")
     ap.add_argument("--op", choices=["quantize", "dequantize", "tensor_scale", "shard"],
                     default="quantize",
                     help="dequantize: time the reverse map on the quantized workload; "
