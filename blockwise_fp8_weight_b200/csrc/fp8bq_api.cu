@@ -132,7 +132,8 @@ bool vector_fits(const fp8bq_desc &D, Variant v) {
     if (D.block_n % vec) return false;
     const int vpr = D.block_n / vec;
     if (!is_pow2(vpr) || vpr > team) return false;
-    if (v == Variant::VecT16) return (int64_t)D.block_m * vpr == team;  // one row-step per block
+    if (v == Variant::VecT16 || v == Variant::VecT32)
+        return (int64_t)D.block_m * vpr == team;  // one row-step per block
     return cdiv(D.block_m, team / vpr) <= slots;
 }
 
@@ -159,7 +160,8 @@ bool halves_aligned(const fp8bq_desc &D) {
 }
 
 Variant vector_variant(const fp8bq_desc &D) {
-    for (Variant v : {Variant::VecT16, Variant::VecT64, Variant::VecTBig})
+    for (Variant v : {Variant::VecT16, Variant::VecT32, Variant::VecT64, Variant::VecT128,
+                      Variant::VecTBig})
         if (vector_fits(D, v)) return v;
     return Variant::Generic;
 }

@@ -153,6 +153,8 @@ enum class Variant : int {
     VecT64 = 2,   // a team of 64 threads per block (<= 512 vectors)
     VecTBig = 3,  // one team per CTA (<= 2048 vectors)
     Tma = 4,
+    VecT32 = 5,   // a team of 32 threads (a warp) per 8 stacked blocks of one row-step each
+    VecT128 = 6,  // a team of 128 threads per block (<= 1024 vectors)
 };
 
 // Launchers (vector and generic: fp8bq_kernels.cu; TMA: fp8bq_tma.cu).  Each
@@ -240,11 +242,17 @@ cudaError_t bounds_record_scale(uint64_t *count, uint64_t *first, bool clear);
 
 // Team geometry used by the vector kernels (host eligibility must agree).
 constexpr int kVecTeamThreads(Variant v, int esize) {
-    return v == Variant::VecT16 ? 16 : v == Variant::VecT64 ? 64 : (esize == 2 ? 256 : 512);
+    return v == Variant::VecT16    ? 16
+           : v == Variant::VecT32  ? 32
+           : v == Variant::VecT64  ? 64
+           : v == Variant::VecT128 ? 128
+                                   : (esize == 2 ? 256 : 512);
 }
 constexpr int kVecSlots(Variant v) { return 8; }
 // Blocks per tile along M: the small-block kernel stacks 8 blocks per tile.
-constexpr int kTileBlocksM(Variant v) { return v == Variant::VecT16 ? 8 : 1; }
+constexpr int kTileBlocksM(Variant v) {
+    return v == Variant::VecT16 || v == Variant::VecT32 ? 8 : 1;
+}
 
 constexpr int kTmaConsumerThreads = 256;
 constexpr int kTmaStageBytes = 32768;

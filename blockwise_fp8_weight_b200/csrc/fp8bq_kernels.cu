@@ -93,6 +93,31 @@ __device__ __forceinline__ uint32_t reduce_scatter8x16(const uint32_t (&m)[8], u
     return max(c, __shfl_xor_sync(mask, c, 1));
 }
 
+// The same over the 32 lanes of a warp: three halving steps (xor 16, 8, 4)
+// and two full ones (xor 2, 1); lane q ends with the team-wide max of slot
+// 4*b4 + 2*b3 + b2, i.e. slot q / 4.
+__device__ __forceinline__ uint32_t reduce_scatter8x32(const uint32_t (&m)[8], int q) {
+    const bool h4 = q & 16, h3 = q & 8, h2 = q & 4;
+    uint32_t a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t send = h4 ? m[j] : m[j + 4];
+        const uint32_t keep = h4 ? m[j + 4] : m[j];
+        a[j] = max(keep, __shfl_xor_sync(0xffffffffu, send, 16));
+    }
+    uint32_t b[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint32_t send = h3 ? a[j] : a[j + 2];
+        const uint32_t keep = h3 ? a[j + 2] : a[j];
+        b[j] = max(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    }
+    const uint32_t send = h2 ? b[0] : b[1];
+    uint32_t c = max(h2 ? b[1] : b[0], __shfl_xor_sync(0xffffffffu, send, 4));
+    c = max(c, __shfl_xor_sync(0xffffffffu, c, 2));
+    return max(c, __shfl_xor_sync(0xffffffffu, c, 1));
+}
+
 // vec_quant_store for a lane's 16 bytes held as two 8-byte halves (rows that
 // are only 8-byte aligned): each half is quantized and stored on its own, the
 // upper one only when hi_ok (it lies inside the row).  Codes: 4 bytes per
@@ -144,7 +169,8 @@ template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES, int
 __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     k_vector(const __grid_constant__ DescPack<MAXD> p) {
     dev::pdl_entry();
-    static_assert(G == 1 || (G == 8 && V == 8 && TEAM == 16), "stacked blocks: 8 over 16 lanes");
+    static_assert(G == 1 || (G == 8 && V == 8 && (TEAM == 16 || TEAM == 32)),
+                  "stacked blocks: 8 over 16 or 32 lanes");
     static_assert(!(HALVES && S > 0), "the cp.async ring takes 16-byte vectors only");
     constexpr int VEC = 16 / ESIZE;
     constexpr int TEAMS = CTA / TEAM;
@@ -219,7 +245,7 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
     };
 
     auto process_slots = [&](const uint4 (&R)[V], const Tile &T) {
-      if constexpr (TEAM == 16 && V == 8) {  // the only stacked-block instantiation
+      if constexpr ((TEAM == 16 || TEAM == 32) && V == 8) {  // the stacked-block instantiations
         const int bm = p.d[0].bm;
         // each slot's maximum as fp32 bits, then integer maxima through the
         // reduce-scatter.  Measured and dropped: keeping the maxima packed as
@@ -233,19 +259,21 @@ __global__ void __launch_bounds__(CTA, (CTA <= 256 ? FP8BQ_VEC_CTAS_PER_SM : 1))
             const uint4 one[1] = {R[i]};
             m[i] = absmax_to_f32_bits<ESIZE>(tile_absmax<ESIZE, 1>(one));
         }
-        // lane q ends with the max of slot q / 2, computes its scale, and the
-        // reciprocal of slot i is fetched from lane 2 i of the team
-        const uint32_t mq = reduce_scatter8x16(m, shfl_mask, lane);
+        // lane q ends with the max of slot q / (TEAM / 8), computes its scale,
+        // and the reciprocal of slot i is fetched from lane (TEAM / 8) i
+        constexpr int LPS = TEAM / 8;  // lanes per slot after the reduce-scatter
+        const uint32_t mq = TEAM == 16 ? reduce_scatter8x16(m, shfl_mask, lane)
+                                       : reduce_scatter8x32(m, lane);
         float s_mine, r_mine;
         dev::block_scale(mq, kEps, s_mine, r_mine);
         const int base = (threadIdx.x & 31) & ~(TEAM - 1);
         float r[V];
 #pragma unroll
-        for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + 2 * i);
+        for (int i = 0; i < V; ++i) r[i] = __shfl_sync(shfl_mask, r_mine, base + LPS * i);
         // slots of blocks below the matrix are neither quantized nor stored
         store_all(R, T, (T.rows + bm - 1) / bm, [&](int i) { return dev::splat2(r[i]); });
-        const int slot = lane >> 1;
-        if ((lane & 1) == 0 && slot * bm < T.rows) store_descale(T, T.sdst + (int64_t)slot * T.gn, s_mine);
+        const int slot = lane / LPS;
+        if (lane % LPS == 0 && slot * bm < T.rows) store_descale(T, T.sdst + (int64_t)slot * T.gn, s_mine);
       }
     };
 
@@ -460,7 +488,7 @@ namespace {
 
 template <int ESIZE, int TEAM, int V, int CTA, int G, int MAXD, bool HALVES>
 cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
-    constexpr int S = HALVES ? 0 : TEAM == 16 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
+    constexpr int S = HALVES ? 0 : TEAM <= 32 ? FP8BQ_VEC_STAGES_T16 : FP8BQ_VEC_STAGES;
     constexpr size_t smem = (size_t)S * V * CTA * 16;
     auto kern = k_vector<ESIZE, TEAM, V, CTA, G, MAXD, HALVES, S>;
     static PerDevice<KernelSetup> setup;
@@ -469,7 +497,7 @@ cudaError_t launch_vector_h(const DescPack<MAXD> &p, cudaStream_t st) {
     // short launches (fewer than FP8BQ_VEC_SHORT_TILES tiles per resident
     // team) take FP8BQ_VEC_WAVES_SHORT waves
     const uint64_t resident_teams = (uint64_t)sm_count() * ks.occ * (CTA / TEAM);
-    const int waves = TEAM == 16 ? FP8BQ_VEC_WAVES_T16
+    const int waves = TEAM <= 32 ? FP8BQ_VEC_WAVES_T16
                       : p.total_tiles < (uint64_t)FP8BQ_VEC_SHORT_TILES * resident_teams
                           ? FP8BQ_VEC_WAVES_SHORT
                           : FP8BQ_VEC_WAVES;
@@ -491,14 +519,18 @@ cudaError_t launch_vector(Variant v, int esize, bool halves, const DescPack<MAXD
     if (esize == 2) {
         switch (v) {
             case Variant::VecT16: return launch_vector_t<2, 16, 8, 256, 8, MAXD>(halves, p, st);
+            case Variant::VecT32: return launch_vector_t<2, 32, 8, 256, 8, MAXD>(halves, p, st);
             case Variant::VecT64: return launch_vector_t<2, 64, 8, 256, 1, MAXD>(halves, p, st);
+            case Variant::VecT128: return launch_vector_t<2, 128, 8, 256, 1, MAXD>(halves, p, st);
             case Variant::VecTBig: return launch_vector_t<2, 256, 8, 256, 1, MAXD>(halves, p, st);
             default: return cudaErrorInvalidValue;
         }
     }
     switch (v) {
         case Variant::VecT16: return launch_vector_t<4, 16, 8, 256, 8, MAXD>(halves, p, st);
+        case Variant::VecT32: return launch_vector_t<4, 32, 8, 256, 8, MAXD>(halves, p, st);
         case Variant::VecT64: return launch_vector_t<4, 64, 8, 256, 1, MAXD>(halves, p, st);
+        case Variant::VecT128: return launch_vector_t<4, 128, 8, 256, 1, MAXD>(halves, p, st);
         case Variant::VecTBig: return launch_vector_t<4, 512, 8, 512, 1, MAXD>(halves, p, st);
         default: return cudaErrorInvalidValue;
     }

@@ -187,6 +187,30 @@ def test_few_row_tensors(shape, block, dtype, ld):
     del owner
 
 
+@pytest.mark.parametrize("shape,block,dtype,ld", [
+    ((1000, 1024), (1, 128), "f32", None),     # 32-lane team, 8 stacked one-row blocks
+    ((777, 1030), (1, 128), "f32", None),      # the same on rows only 8-byte aligned
+    ((1000, 1024), (2, 128), "bf16", None),    # 32-lane team: two rows of 16 vectors
+    ((600, 1024), (1, 256), "bf16", None),     # 32-lane team: one row of 32 vectors
+    ((1000, 1024), (64, 64), "f32", None),     # 128-thread team
+    ((1000, 1024), (128, 64), "bf16", 1088),   # 128-thread team, padded rows
+])
+def test_stacked_and_mid_size_teams(shape, block, dtype, ld):
+    """Block shapes served by the 32-lane stacked-block team and the 128-thread
+    team: every code and descale against the oracle, on every path."""
+    M, N = shape
+    sp = TensorSpec(f"team.{M}x{N}.b{block}.{dtype}", M, N, block=block, dtype=dtype, ld=ld,
+                    seed=79, tensor_id=M + block[0] * 7 + block[1], dist=DIST_STUDENT_T3,
+                    row_lognormal_sigma=1.0)
+    x = W.materialize(sp)
+    owner, ptr = to_device(x)
+    want = oracle_expected(sp, x)
+    for path in PATHS.values():
+        (o,) = run([sp], [ptr], path)
+        assert_same(sp, o.result(), want)
+    del owner
+
+
 def test_all_zero_and_one_element_blocks():
     sp = TensorSpec("zeros", 200, 264, seed=0)
     x = np.zeros(sp.numel_storage, dtype=np.uint16)
