@@ -14,7 +14,9 @@
  *     descale  = s
  *
  * where e4m3fn() rounds to nearest, ties to even, saturating, and keeps the
- * sign of a result that rounds to zero; eps = 1e-10f.  The pages print the
+ * sign of a result that rounds to zero; eps = 1e-10f.  (The kernels reach the
+ * two correctly rounded quotients without division instructions; the values
+ * are those of IEEE division.)  The pages print the
  * eps floor but not its value; 1e-10f is this library's reading.  The result
  * is unique bit for bit: there is no summation, and max is order independent.
  *
